@@ -1,0 +1,213 @@
+/*
+ * pa.h -- C ABI of the B200 paged-KV-cache decode library (libpagedattn.so).
+ *
+ * What it computes. vLLM's PagedAttention keeps each sequence's KV cache in
+ * fixed 16-token blocks scattered through one physical pool; a per-sequence
+ * block table maps logical block (position // block_size) to physical block,
+ * and a Block Manager hands blocks out and takes them back in O(1) with a free
+ * list (vLLM notes page, "PagedAttention": Block Manager and Cache Engine;
+ * "vLLM 前世今生" section 3.2: 16-token blocks, non-contiguous physical blocks,
+ * block table, blocks shared by several sequences). This library provides the
+ * decode-step hot path of that design on one GPU:
+ *   - pa_reshape_and_cache: scatter each new token's K and V into its slot
+ *     (the Cache Engine's write side);
+ *   - pa_decode: one query token per sequence attends over its whole paged
+ *     context, out = softmax(scale * q K^T) V, reading K/V through the block
+ *     table (the PagedAttention kernel);
+ *   - a host-side free-list block allocator with reference counts, used to
+ *     build block tables and to share prefix blocks between sequences.
+ *
+ * Conventions (all calls).
+ *   - Device tensors are caller-owned (PyTorch or any allocator); the library
+ *     never allocates, frees or synchronises on pa_reshape_and_cache/pa_decode.
+ *     Work is enqueued on the caller's stream (a cudaStream_t passed as void*;
+ *     NULL = the legacy default stream). Calls return after enqueueing.
+ *   - Host-side validation runs before any launch and returns a negative
+ *     pa_status without touching device memory; pa_last_error() then gives a
+ *     one-line reason (thread-local). A launch failure returns PA_ERR_CUDA.
+ *   - Conditions only the device can see (a block id or slot outside the pool,
+ *     a context longer than max_context_len, a pipeline wait that timed out)
+ *     never fault: the offending page or token is skipped and a bit is OR-ed
+ *     into an error word (PA_DEVERR_*), the caller's if given, else the
+ *     library's own, read with pa_read_device_error().
+ *   - Block size is fixed at 16 tokens.
+ *
+ * Pool layout. Each cache (K and V separately) is a contiguous tensor
+ * [num_blocks, num_kv_heads, 16, head_dim]: one (block, head) page is one
+ * contiguous run of 16 * head_dim elements. Slot s of the pool is token row
+ * s % 16 of physical block s / 16.
+ */
+#ifndef PAGED_KV_CACHE_PA_H
+#define PAGED_KV_CACHE_PA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define PA_BLOCK_SIZE 16
+
+typedef enum pa_status {
+  PA_OK = 0,
+  PA_ERR_INVALID_ARG = -1, /* shape, dtype, stride, alignment or value outside the contract  */
+  PA_ERR_UNSUPPORTED = -2, /* valid but not built: head_dim, group size or dtype combination  */
+  PA_ERR_WORKSPACE = -3,   /* split partitions need a workspace that was missing or too small */
+  PA_ERR_CUDA = -4,        /* a CUDA runtime call or launch failed                            */
+  PA_ERR_EXHAUSTED = -5,   /* allocator: no free block                                        */
+  PA_ERR_BAD_BLOCK = -6    /* allocator: block id out of range, or not allocated              */
+} pa_status;
+
+/* Element types of pa_tensor.dtype. PA_E4M3 is OCP FP8 E4M3 ("fn": no infinities, max 448). */
+typedef enum pa_dtype { PA_F16 = 0, PA_BF16 = 1, PA_E4M3 = 2, PA_I32 = 3, PA_I64 = 4, PA_F32 = 5 } pa_dtype;
+
+/* Device-side error bits (OR-ed into the error word). */
+#define PA_DEVERR_BAD_BLOCK 1u   /* a block-table entry read for a valid position is outside [0, num_blocks) */
+#define PA_DEVERR_BAD_SLOT 2u    /* a slot_mapping entry is < -1 or >= num_blocks * 16                       */
+#define PA_DEVERR_TIMEOUT 4u     /* a wait for an asynchronous page copy exceeded its bound                  */
+#define PA_DEVERR_CTX_RANGE 8u   /* context_lens[s] > max_context_len (or > 16 * block-table width)          */
+
+/* A strided view of caller-owned memory. Strides are in elements, not bytes.
+ * Only the first ndim entries of shape/stride are read. The pointer is a
+ * device pointer for pa_reshape_and_cache/pa_decode. */
+typedef struct pa_tensor {
+  void* data;
+  int32_t dtype; /* pa_dtype */
+  int32_t ndim;
+  int64_t shape[4];
+  int64_t stride[4];
+} pa_tensor;
+
+/* Optional knobs of pa_decode. Pass NULL for all defaults; a zeroed struct is
+ * NOT the default (scales would be 0): call pa_decode_opts_init first. */
+typedef struct pa_decode_opts {
+  float k_scale;            /* e4m3 caches: stored code * k_scale is the key value; 1 otherwise      */
+  float v_scale;            /* same for values                                                          */
+  int32_t max_context_len;  /* host-known bound on context_lens (sizes the grid without a device read);
+                               0 = 16 * block_tables.shape[1]                                           */
+  int32_t partition_tokens; /* split each context into partitions of this many tokens (multiple of 16,
+                               <= 2048), merged by a second kernel; 0 = library's choice
+                               (pa_decode_partition_tokens)                                            */
+  void* workspace;          /* device scratch for split partitions, >= pa_decode_workspace_bytes, 256-B
+                               aligned; may be NULL when no split happens                               */
+  size_t workspace_bytes;
+  int32_t kernel;           /* -1 = choose; 0 = CUDA-core FMA kernel; 1 = tensor-core (mma) kernel     */
+  int32_t* error_word;      /* device int32 that receives PA_DEVERR_* bits; NULL = library's own word  */
+} pa_decode_opts;
+
+/* Fill opts with the defaults (scales 1, everything else automatic). */
+void pa_decode_opts_init(pa_decode_opts* opts);
+
+/*
+ * pa_reshape_and_cache -- write new tokens' K and V into the paged pool.
+ *   key, value    [T, Hkv, D] device, dtype F16 or BF16, last stride 1, 16-B aligned rows.
+ *   slot_mapping  [T] device I64: slot of token t, or -1 to skip it.
+ *   k_cache, v_cache  [num_blocks, Hkv, 16, D] contiguous, same dtype as key (16-bit caches: the
+ *                 bits are copied unchanged) or E4M3 (code = e4m3_rn_satfinite(float32(x) *
+ *                 float32(1 / scale)), 1/scale formed once in float32 on the host).
+ *   k_scale, v_scale  dequantisation scales of an E4M3 cache (> 0, finite); ignored otherwise.
+ *   Slots outside [-1, num_blocks * 16) are skipped and set PA_DEVERR_BAD_SLOT in the library's
+ *   error word. Untouched slots keep their bytes. Two tokens with the same slot race.
+ * Source: vLLM notes page, "PagedAttention / Cache Engine" (the engine writes a position's data
+ * into its page). T == 0 is a no-op.
+ */
+int pa_reshape_and_cache(const pa_tensor* key, const pa_tensor* value, const pa_tensor* slot_mapping,
+                         pa_tensor* k_cache, pa_tensor* v_cache, float k_scale, float v_scale, void* stream);
+
+/*
+ * pa_decode -- one decode step of paged attention.
+ *   out           [B, Hq, D] device, same dtype as q, last stride 1, 16-B aligned rows.
+ *   q             [B, Hq, D] device F16 or BF16 (F16 with an F16 cache, BF16 with a BF16 cache,
+ *                 either with an E4M3 cache; with E4M3 q must lie within the f16 range).
+ *   k_cache, v_cache  [num_blocks, Hkv, 16, D] contiguous, dtype F16, BF16 or E4M3 (both the same).
+ *   block_tables  [B, max_blocks] device I32 (last stride 1): physical block of logical block j of
+ *                 sequence s. Entries at j >= ceil(context_lens[s] / 16) are never read.
+ *   context_lens  [B] device I32: tokens of sequence s (already including the token written this
+ *                 step by pa_reshape_and_cache). 0 gives an all-zero output row.
+ *   scale         multiplies q.k before the softmax (typically 1/sqrt(D)).
+ *   num_kv_heads  Hkv; must equal k_cache.shape[1] and divide Hq. Query head h reads KV head
+ *                 h / (Hq / Hkv). Supported: D in {64, 128} (E4M3: 128), Hq / Hkv <= 16.
+ * out[s, h, :] = sum_t softmax_t(scale * q[s, h] . K[s, t]) V[s, t], K[s, t] being row t % 16 of
+ * page (block_tables[s][t / 16], h / G); accumulation in float32, result rounded to nearest even.
+ * The result depends only on logical positions, never on which physical blocks hold them.
+ * Source: vLLM notes page, "PagedAttention" (page of a position = position // block_size) and
+ * "内核优化" (kernels section: the PagedAttention kernel, GQA and MQA kernels); "vLLM 前世今生"
+ * section 3.2.
+ */
+int pa_decode(pa_tensor* out, const pa_tensor* q, const pa_tensor* k_cache, const pa_tensor* v_cache,
+              const pa_tensor* block_tables, const pa_tensor* context_lens, float scale, int32_t num_kv_heads,
+              const pa_decode_opts* opts, void* stream);
+
+/* Partition size pa_decode uses when opts->partition_tokens == 0 and a workspace is given
+ * (0 = no split). Host only. */
+int32_t pa_decode_partition_tokens(int32_t num_seqs, int32_t num_kv_heads, int32_t max_context_len);
+
+/* Workspace bytes pa_decode needs for these sizes (0 when no split happens). partition_tokens 0
+ * applies the library's choice. Host only. */
+size_t pa_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t head_dim,
+                                 int32_t max_context_len, int32_t partition_tokens);
+
+/* Static string for a pa_status value. */
+const char* pa_status_string(int status);
+
+/* Reason for the last non-OK return on this thread ("" if none). */
+const char* pa_last_error(void);
+
+/* Synchronise the current device, copy the library's own device error word (PA_DEVERR_* bits)
+ * into *bits and, if clear != 0, reset it to 0. Not for hot paths. */
+int pa_read_device_error(uint32_t* bits, int clear);
+
+/* Library version, "major.minor.patch". */
+const char* pa_version(void);
+
+/* ---------------------------------------------------------------------------------------------
+ * Host block allocator: free list of physical block ids with reference counts.
+ * Source: vLLM notes page, "PagedAttention / Block Manager" (O(1) allocation and release with a
+ * free list); "vLLM 前世今生" section 3.2 (blocks allocated on demand, freed when a sequence
+ * finishes, several sequences may point at one physical block).
+ * alloc pops the top of a stack of free ids; the release of a block's last reference pushes it
+ * back on top. Every call is O(1) (the _n variants O(n)). Not thread-safe: one allocator per
+ * thread, or external locking. No GPU involved.
+ * ------------------------------------------------------------------------------------------- */
+typedef struct pa_allocator pa_allocator;
+
+/* New allocator over block ids [0, num_blocks). initial_order (nullable, a permutation of
+ * [0, num_blocks)) is the order the first allocations come out in; NULL means 0, 1, 2, ...
+ * Returns NULL on a bad argument (pa_last_error says why) or out of host memory. */
+pa_allocator* pa_allocator_create(int32_t num_blocks, const int32_t* initial_order);
+void pa_allocator_destroy(pa_allocator* a);
+
+/* A free block id with refcount 1, or PA_ERR_EXHAUSTED. */
+int32_t pa_block_alloc(pa_allocator* a);
+/* Add a reference to an allocated block (share it). PA_ERR_BAD_BLOCK if not allocated. */
+int pa_block_incref(pa_allocator* a, int32_t block);
+/* Drop a reference; at 0 the block returns to the free list. PA_ERR_BAD_BLOCK if not allocated. */
+int pa_block_free(pa_allocator* a, int32_t block);
+/* Reference count of a block (0 = free), or PA_ERR_BAD_BLOCK for an id outside the pool. */
+int32_t pa_block_refcount(const pa_allocator* a, int32_t block);
+int32_t pa_allocator_num_free(const pa_allocator* a);
+int32_t pa_allocator_num_blocks(const pa_allocator* a);
+
+/* Allocate n blocks into out[0..n) all-or-nothing: PA_ERR_EXHAUSTED (nothing taken) if fewer
+ * than n are free. */
+int pa_blocks_alloc_n(pa_allocator* a, int32_t n, int32_t* out);
+/* incref / free each of blocks[0..n); stops at the first bad id and returns its error. */
+int pa_blocks_incref_n(pa_allocator* a, int32_t n, const int32_t* blocks);
+int pa_blocks_free_n(pa_allocator* a, int32_t n, const int32_t* blocks);
+
+/* Host helper: slot of each (sequence, position) pair, slot = bt[seq][pos / 16] * 16 + pos % 16.
+ *   block_tables  host I32, num_seqs rows of row_stride elements, max_blocks valid entries each.
+ *   token_seq, token_pos, slots_out  host arrays of num_tokens entries.
+ * PA_ERR_INVALID_ARG if a sequence or logical block is out of range or the entry is negative.
+ * Source: vLLM notes page, "PagedAttention / Cache Engine" (page = position // block_size); the
+ * in-block offset position % 16 is the plain reading of a 16-token page. */
+int pa_slots_for_positions(const int32_t* block_tables, int64_t row_stride, int32_t num_seqs, int32_t max_blocks,
+                           const int32_t* token_seq, const int32_t* token_pos, int64_t num_tokens,
+                           int64_t* slots_out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGED_KV_CACHE_PA_H */

@@ -1,0 +1,131 @@
+// Host-side block allocator: a stack of free physical block ids plus reference counts.
+//
+// Source: vLLM notes page, "PagedAttention / Block Manager": pages are handed out when a request
+// needs them and marked reusable when it no longer does, with a free list (or a bitmap) so that
+// both operations are O(1). "vLLM 前世今生" section 3.2: several sequences may point at one
+// physical block (parallel sampling, beam search, shared prefixes), so a block carries a count of
+// the sequences that reference it and returns to the free list when the last one lets go.
+//
+// alloc pops the top of the stack; freeing the last reference pushes the block back on top, so the
+// block released most recently is reused first (warm in L2). No GPU is involved.
+#include <cstdint>
+#include <new>
+#include <vector>
+
+#include "../../include/pa.h"
+
+struct pa_allocator {
+  std::vector<int32_t> stack;  // free ids; top = back
+  std::vector<int32_t> ref;    // 0 = free
+};
+
+extern "C" {
+
+pa_allocator* pa_allocator_create(int32_t num_blocks, const int32_t* initial_order) {
+  if (num_blocks <= 0) return nullptr;
+  pa_allocator* a = new (std::nothrow) pa_allocator;
+  if (!a) return nullptr;
+  try {
+    a->ref.assign(static_cast<size_t>(num_blocks), 0);
+    a->stack.resize(static_cast<size_t>(num_blocks));
+  } catch (...) {
+    delete a;
+    return nullptr;
+  }
+  if (initial_order) {
+    // Must be a permutation of [0, num_blocks); pops come out in this order.
+    std::vector<char> seen(static_cast<size_t>(num_blocks), 0);
+    for (int32_t i = 0; i < num_blocks; ++i) {
+      const int32_t b = initial_order[i];
+      if (b < 0 || b >= num_blocks || seen[b]) {
+        delete a;
+        return nullptr;
+      }
+      seen[b] = 1;
+      a->stack[num_blocks - 1 - i] = b;
+    }
+  } else {
+    for (int32_t i = 0; i < num_blocks; ++i) a->stack[num_blocks - 1 - i] = i;
+  }
+  return a;
+}
+
+void pa_allocator_destroy(pa_allocator* a) { delete a; }
+
+int32_t pa_block_alloc(pa_allocator* a) {
+  if (!a) return PA_ERR_INVALID_ARG;
+  if (a->stack.empty()) return PA_ERR_EXHAUSTED;
+  const int32_t b = a->stack.back();
+  a->stack.pop_back();
+  a->ref[b] = 1;
+  return b;
+}
+
+int pa_block_incref(pa_allocator* a, int32_t b) {
+  if (!a) return PA_ERR_INVALID_ARG;
+  if (b < 0 || b >= static_cast<int32_t>(a->ref.size()) || a->ref[b] == 0) return PA_ERR_BAD_BLOCK;
+  if (a->ref[b] == INT32_MAX) return PA_ERR_INVALID_ARG;
+  ++a->ref[b];
+  return PA_OK;
+}
+
+int pa_block_free(pa_allocator* a, int32_t b) {
+  if (!a) return PA_ERR_INVALID_ARG;
+  if (b < 0 || b >= static_cast<int32_t>(a->ref.size()) || a->ref[b] == 0) return PA_ERR_BAD_BLOCK;
+  if (--a->ref[b] == 0) a->stack.push_back(b);
+  return PA_OK;
+}
+
+int32_t pa_block_refcount(const pa_allocator* a, int32_t b) {
+  if (!a) return PA_ERR_INVALID_ARG;
+  if (b < 0 || b >= static_cast<int32_t>(a->ref.size())) return PA_ERR_BAD_BLOCK;
+  return a->ref[b];
+}
+
+int32_t pa_allocator_num_free(const pa_allocator* a) { return a ? static_cast<int32_t>(a->stack.size()) : PA_ERR_INVALID_ARG; }
+
+int32_t pa_allocator_num_blocks(const pa_allocator* a) { return a ? static_cast<int32_t>(a->ref.size()) : PA_ERR_INVALID_ARG; }
+
+int pa_blocks_alloc_n(pa_allocator* a, int32_t n, int32_t* out) {
+  if (!a || n < 0 || (n > 0 && !out)) return PA_ERR_INVALID_ARG;
+  if (static_cast<size_t>(n) > a->stack.size()) return PA_ERR_EXHAUSTED;
+  for (int32_t i = 0; i < n; ++i) out[i] = pa_block_alloc(a);
+  return PA_OK;
+}
+
+int pa_blocks_incref_n(pa_allocator* a, int32_t n, const int32_t* blocks) {
+  if (!a || n < 0 || (n > 0 && !blocks)) return PA_ERR_INVALID_ARG;
+  for (int32_t i = 0; i < n; ++i) {
+    const int r = pa_block_incref(a, blocks[i]);
+    if (r != PA_OK) return r;
+  }
+  return PA_OK;
+}
+
+int pa_blocks_free_n(pa_allocator* a, int32_t n, const int32_t* blocks) {
+  if (!a || n < 0 || (n > 0 && !blocks)) return PA_ERR_INVALID_ARG;
+  for (int32_t i = 0; i < n; ++i) {
+    const int r = pa_block_free(a, blocks[i]);
+    if (r != PA_OK) return r;
+  }
+  return PA_OK;
+}
+
+int pa_slots_for_positions(const int32_t* bt, int64_t row_stride, int32_t num_seqs, int32_t max_blocks,
+                           const int32_t* token_seq, const int32_t* token_pos, int64_t num_tokens, int64_t* out) {
+  if (num_tokens < 0 || (num_tokens > 0 && (!bt || !token_seq || !token_pos || !out)) || num_seqs < 0 ||
+      max_blocks < 0 || row_stride < max_blocks)
+    return PA_ERR_INVALID_ARG;
+  for (int64_t i = 0; i < num_tokens; ++i) {
+    const int32_t s = token_seq[i], pos = token_pos[i];
+    if (s < 0 || s >= num_seqs || pos < 0) return PA_ERR_INVALID_ARG;
+    const int32_t j = pos / PA_BLOCK_SIZE;
+    if (j >= max_blocks) return PA_ERR_INVALID_ARG;
+    const int32_t b = bt[static_cast<int64_t>(s) * row_stride + j];
+    if (b < 0) return PA_ERR_INVALID_ARG;
+    out[i] = static_cast<int64_t>(b) * PA_BLOCK_SIZE + pos % PA_BLOCK_SIZE;
+  }
+  return PA_OK;
+}
+
+}  // extern "C"

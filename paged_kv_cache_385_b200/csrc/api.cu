@@ -1,0 +1,400 @@
+// C-ABI entry points of libpagedattn: argument validation, TMA descriptor encoding, dispatch.
+// Host code only; the kernels live in decode.cu and cache.cu.
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "../../include/pa.h"
+#include "internal.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(int status, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return status;
+}
+
+int ok() {
+  g_last_error.clear();
+  return PA_OK;
+}
+
+int elem_bytes(int dtype) {
+  switch (dtype) {
+    case PA_F16:
+    case PA_BF16:
+      return 2;
+    case PA_E4M3:
+      return 1;
+    case PA_I32:
+    case PA_F32:
+      return 4;
+    case PA_I64:
+      return 8;
+    default:
+      return 0;
+  }
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+bool is_contiguous(const pa_tensor* t) {
+  int64_t expect = 1;
+  for (int i = t->ndim - 1; i >= 0; --i) {
+    if (t->shape[i] != 1 && t->stride[i] != expect) return false;
+    expect *= t->shape[i];
+  }
+  return true;
+}
+
+const char* dtype_name(int d) {
+  switch (d) {
+    case PA_F16: return "F16";
+    case PA_BF16: return "BF16";
+    case PA_E4M3: return "E4M3";
+    case PA_I32: return "I32";
+    case PA_I64: return "I64";
+    case PA_F32: return "F32";
+    default: return "?";
+  }
+}
+
+// Checks common to every tensor argument.
+int check_tensor(const pa_tensor* t, const char* name, int ndim) {
+  if (!t) return fail(PA_ERR_INVALID_ARG, "%s is NULL", name);
+  if (t->ndim != ndim) return fail(PA_ERR_INVALID_ARG, "%s: ndim %d, expected %d", name, t->ndim, ndim);
+  if (elem_bytes(t->dtype) == 0) return fail(PA_ERR_INVALID_ARG, "%s: unknown dtype %d", name, t->dtype);
+  for (int i = 0; i < ndim; ++i)
+    if (t->shape[i] < 0) return fail(PA_ERR_INVALID_ARG, "%s: negative shape[%d]", name, i);
+  return PA_OK;
+}
+
+// ---- TMA descriptor encoding -----------------------------------------------------------------
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// The pool [NB, Hkv, 16, D] viewed as a 2-D tensor [NB * Hkv * 16 rows, D], loaded in boxes of
+// 16 rows x 128 bytes with the 128-byte swizzle.
+int encode_pool_map(CUtensorMap* map, const pa_tensor* cache, int esz) {
+  auto fn = encode_fn();
+  if (!fn) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const int64_t D = cache->shape[3];
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(D),
+                              static_cast<cuuint64_t>(cache->shape[0] * cache->shape[1] * 16)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(D * esz)};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / esz), 16};
+  const cuuint32_t estr[2] = {1, 1};
+  CUtensorMapDataType dt = esz == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                    : (cache->dtype == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                               : CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
+  CUresult r = fn(map, dt, 2, cache->data, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return PA_OK;
+}
+
+uint32_t* library_error_word() {
+  static uint32_t* words[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return nullptr;
+  if (dev >= 64) return pa::decode_error_word();
+  if (!words[dev]) words[dev] = pa::decode_error_word();
+  return words[dev];
+}
+
+int32_t auto_partition_tokens(int32_t max_ctx) { return max_ctx > 512 ? 512 : 0; }
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Layout of the split-partition workspace: acc [B, Hq, P, D] floats, then (m, l) [B, Hq, P, 2].
+size_t workspace_layout(int64_t B, int64_t Hq, int64_t D, int64_t P, size_t* ml_offset) {
+  const size_t acc = round_up(static_cast<size_t>(B * Hq * P * D) * sizeof(float), 256);
+  const size_t ml = round_up(static_cast<size_t>(B * Hq * P * 2) * sizeof(float), 256);
+  if (ml_offset) *ml_offset = acc;
+  return acc + ml;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* pa_version(void) { return "0.1.0"; }
+
+const char* pa_status_string(int status) {
+  switch (status) {
+    case PA_OK: return "ok";
+    case PA_ERR_INVALID_ARG: return "invalid argument";
+    case PA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case PA_ERR_WORKSPACE: return "workspace missing or too small";
+    case PA_ERR_CUDA: return "CUDA error";
+    case PA_ERR_EXHAUSTED: return "no free block";
+    case PA_ERR_BAD_BLOCK: return "bad block id";
+    default: return "unknown status";
+  }
+}
+
+const char* pa_last_error(void) { return g_last_error.c_str(); }
+
+void pa_decode_opts_init(pa_decode_opts* o) {
+  if (!o) return;
+  std::memset(o, 0, sizeof(*o));
+  o->k_scale = 1.0f;
+  o->v_scale = 1.0f;
+  o->kernel = -1;
+}
+
+int32_t pa_decode_partition_tokens(int32_t num_seqs, int32_t num_kv_heads, int32_t max_context_len) {
+  (void)num_seqs;
+  (void)num_kv_heads;
+  return auto_partition_tokens(max_context_len);
+}
+
+size_t pa_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t head_dim, int32_t max_context_len,
+                                 int32_t partition_tokens) {
+  if (num_seqs <= 0 || num_q_heads <= 0 || head_dim <= 0 || max_context_len <= 0) return 0;
+  const int32_t pt = partition_tokens > 0 ? partition_tokens : auto_partition_tokens(max_context_len);
+  if (pt <= 0) return 0;
+  const int64_t P = (static_cast<int64_t>(max_context_len) + pt - 1) / pt;
+  if (P <= 1) return 0;
+  return workspace_layout(num_seqs, num_q_heads, head_dim, P, nullptr);
+}
+
+int pa_read_device_error(uint32_t* bits, int clear) {
+  if (!bits) return fail(PA_ERR_INVALID_ARG, "bits is NULL");
+  cudaError_t e = pa::read_and_clear_error_word(bits, clear);
+  if (e != cudaSuccess) return fail(PA_ERR_CUDA, "reading the device error word: %s", cudaGetErrorString(e));
+  return ok();
+}
+
+int pa_reshape_and_cache(const pa_tensor* key, const pa_tensor* value, const pa_tensor* slot_mapping,
+                         pa_tensor* k_cache, pa_tensor* v_cache, float k_scale, float v_scale, void* stream) {
+  int st;
+  if ((st = check_tensor(key, "key", 3)) || (st = check_tensor(value, "value", 3)) ||
+      (st = check_tensor(slot_mapping, "slot_mapping", 1)) || (st = check_tensor(k_cache, "k_cache", 4)) ||
+      (st = check_tensor(v_cache, "v_cache", 4)))
+    return st;
+  const int64_t T = key->shape[0], Hkv = key->shape[1], D = key->shape[2];
+  if (key->dtype != PA_F16 && key->dtype != PA_BF16)
+    return fail(PA_ERR_INVALID_ARG, "key dtype %s; expected F16 or BF16", dtype_name(key->dtype));
+  if (value->dtype != key->dtype) return fail(PA_ERR_INVALID_ARG, "value dtype differs from key dtype");
+  for (int i = 0; i < 3; ++i)
+    if (value->shape[i] != key->shape[i]) return fail(PA_ERR_INVALID_ARG, "value shape differs from key shape");
+  if (slot_mapping->dtype != PA_I64) return fail(PA_ERR_INVALID_ARG, "slot_mapping dtype must be I64");
+  if (slot_mapping->shape[0] != T) return fail(PA_ERR_INVALID_ARG, "slot_mapping has %lld entries, key has %lld tokens",
+                                               (long long)slot_mapping->shape[0], (long long)T);
+  if (T > 0x7fffffff) return fail(PA_ERR_INVALID_ARG, "too many tokens (%lld)", (long long)T);
+  if (k_cache->dtype != v_cache->dtype) return fail(PA_ERR_INVALID_ARG, "k_cache and v_cache dtypes differ");
+  const int cd = k_cache->dtype;
+  if (cd != key->dtype && cd != PA_E4M3)
+    return fail(PA_ERR_INVALID_ARG, "cache dtype %s does not match key dtype %s (or E4M3)", dtype_name(cd),
+                dtype_name(key->dtype));
+  for (int i = 0; i < 4; ++i)
+    if (v_cache->shape[i] != k_cache->shape[i]) return fail(PA_ERR_INVALID_ARG, "v_cache shape differs from k_cache");
+  if (k_cache->shape[1] != Hkv || k_cache->shape[2] != PA_BLOCK_SIZE || k_cache->shape[3] != D)
+    return fail(PA_ERR_INVALID_ARG, "cache shape must be [num_blocks, %lld, 16, %lld]", (long long)Hkv, (long long)D);
+  if (!is_contiguous(k_cache) || !is_contiguous(v_cache)) return fail(PA_ERR_INVALID_ARG, "caches must be contiguous");
+  if (D % 8 != 0 || D <= 0) return fail(PA_ERR_UNSUPPORTED, "head_dim %lld is not a multiple of 8", (long long)D);
+  if (T == 0) return ok();
+  if (key->stride[2] != 1 || value->stride[2] != 1) return fail(PA_ERR_INVALID_ARG, "key/value last stride must be 1");
+  if (!aligned(key->data, 16) || !aligned(value->data, 16) || key->stride[0] % 8 || key->stride[1] % 8 ||
+      value->stride[0] % 8 || value->stride[1] % 8)
+    return fail(PA_ERR_INVALID_ARG, "key/value rows must be 16-byte aligned");
+  if (slot_mapping->stride[0] != 1) return fail(PA_ERR_INVALID_ARG, "slot_mapping must be contiguous");
+  if (!aligned(k_cache->data, 16) || !aligned(v_cache->data, 16))
+    return fail(PA_ERR_INVALID_ARG, "caches must be 16-byte aligned");
+  if (!key->data || !value->data || !slot_mapping->data || !k_cache->data || !v_cache->data)
+    return fail(PA_ERR_INVALID_ARG, "NULL data pointer");
+
+  pa::CacheParams p{};
+  p.key = key->data;
+  p.value = value->data;
+  p.k_stride_t = key->stride[0];
+  p.k_stride_h = key->stride[1];
+  p.v_stride_t = value->stride[0];
+  p.v_stride_h = value->stride[1];
+  p.slots = static_cast<const int64_t*>(slot_mapping->data);
+  p.k_cache = k_cache->data;
+  p.v_cache = v_cache->data;
+  p.num_tokens = T;
+  p.num_kv_heads = static_cast<int32_t>(Hkv);
+  p.head_dim = static_cast<int32_t>(D);
+  p.num_slots = k_cache->shape[0] * PA_BLOCK_SIZE;
+  p.k_inv_scale = 1.0f;
+  p.v_inv_scale = 1.0f;
+  if (cd == PA_E4M3) {
+    if (!(std::isfinite(k_scale) && k_scale > 0.f && std::isfinite(v_scale) && v_scale > 0.f))
+      return fail(PA_ERR_INVALID_ARG, "E4M3 cache scales must be finite and > 0");
+    volatile float one = 1.0f;  // keep the reciprocal an IEEE float32 division
+    p.k_inv_scale = one / k_scale;
+    p.v_inv_scale = one / v_scale;
+  }
+  p.err = library_error_word();
+  if (!p.err) return fail(PA_ERR_CUDA, "no device error word (no current CUDA device?)");
+  const pa::KvType kv = cd == PA_E4M3 ? pa::KvType::E4M3 : (cd == PA_BF16 ? pa::KvType::BF16 : pa::KvType::F16);
+  cudaError_t e = pa::launch_reshape_and_cache(key->dtype == PA_BF16, kv, p, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(PA_ERR_CUDA, "reshape_and_cache launch: %s", cudaGetErrorString(e));
+  return ok();
+}
+
+int pa_decode(pa_tensor* out, const pa_tensor* q, const pa_tensor* k_cache, const pa_tensor* v_cache,
+              const pa_tensor* block_tables, const pa_tensor* context_lens, float scale, int32_t num_kv_heads,
+              const pa_decode_opts* opts_in, void* stream) {
+  pa_decode_opts opts;
+  pa_decode_opts_init(&opts);
+  if (opts_in) opts = *opts_in;
+  int st;
+  if ((st = check_tensor(out, "out", 3)) || (st = check_tensor(q, "q", 3)) || (st = check_tensor(k_cache, "k_cache", 4)) ||
+      (st = check_tensor(v_cache, "v_cache", 4)) || (st = check_tensor(block_tables, "block_tables", 2)) ||
+      (st = check_tensor(context_lens, "context_lens", 1)))
+    return st;
+  const int64_t B = q->shape[0], Hq = q->shape[1], D = q->shape[2];
+  if (q->dtype != PA_F16 && q->dtype != PA_BF16) return fail(PA_ERR_INVALID_ARG, "q dtype must be F16 or BF16");
+  if (out->dtype != q->dtype) return fail(PA_ERR_INVALID_ARG, "out dtype differs from q dtype");
+  for (int i = 0; i < 3; ++i)
+    if (out->shape[i] != q->shape[i]) return fail(PA_ERR_INVALID_ARG, "out shape differs from q shape");
+  if (k_cache->dtype != v_cache->dtype) return fail(PA_ERR_INVALID_ARG, "k_cache and v_cache dtypes differ");
+  const int cd = k_cache->dtype;
+  if (cd != PA_F16 && cd != PA_BF16 && cd != PA_E4M3) return fail(PA_ERR_INVALID_ARG, "cache dtype must be F16, BF16 or E4M3");
+  if (cd != PA_E4M3 && cd != q->dtype)
+    return fail(PA_ERR_INVALID_ARG, "a %s cache needs a %s query (got %s)", dtype_name(cd), dtype_name(cd),
+                dtype_name(q->dtype));
+  for (int i = 0; i < 4; ++i)
+    if (v_cache->shape[i] != k_cache->shape[i]) return fail(PA_ERR_INVALID_ARG, "v_cache shape differs from k_cache");
+  if (num_kv_heads <= 0 || k_cache->shape[1] != num_kv_heads)
+    return fail(PA_ERR_INVALID_ARG, "num_kv_heads %d does not match k_cache.shape[1] = %lld", num_kv_heads,
+                (long long)k_cache->shape[1]);
+  if (k_cache->shape[2] != PA_BLOCK_SIZE || k_cache->shape[3] != D)
+    return fail(PA_ERR_INVALID_ARG, "cache shape must be [num_blocks, Hkv, 16, %lld]", (long long)D);
+  if (!is_contiguous(k_cache) || !is_contiguous(v_cache)) return fail(PA_ERR_INVALID_ARG, "caches must be contiguous");
+  if (Hq % num_kv_heads != 0) return fail(PA_ERR_INVALID_ARG, "num_q_heads %lld is not a multiple of num_kv_heads %d",
+                                          (long long)Hq, num_kv_heads);
+  if (block_tables->dtype != PA_I32 || block_tables->shape[0] != B)
+    return fail(PA_ERR_INVALID_ARG, "block_tables must be I32 [num_seqs, max_blocks]");
+  if (context_lens->dtype != PA_I32 || context_lens->shape[0] != B)
+    return fail(PA_ERR_INVALID_ARG, "context_lens must be I32 [num_seqs]");
+  if (!(std::isfinite(scale))) return fail(PA_ERR_INVALID_ARG, "scale must be finite");
+  const int64_t G = Hq / num_kv_heads;
+  if (B == 0 || Hq == 0) return ok();
+  const int64_t NB = k_cache->shape[0];
+  if (NB <= 0) return fail(PA_ERR_INVALID_ARG, "empty pool");
+  if (NB * num_kv_heads * 16 > 0x7fffffffLL) return fail(PA_ERR_UNSUPPORTED, "pool too large (rows exceed 2^31)");
+  if (B > 65535 || num_kv_heads > 65535) return fail(PA_ERR_UNSUPPORTED, "num_seqs and num_kv_heads must be <= 65535");
+  if (G > 16) return fail(PA_ERR_UNSUPPORTED, "query group %lld > 16", (long long)G);
+  if (q->stride[2] != 1 || out->stride[2] != 1) return fail(PA_ERR_INVALID_ARG, "q/out last stride must be 1");
+  if (!aligned(q->data, 16) || !aligned(out->data, 16) || q->stride[0] % 8 || q->stride[1] % 8 || out->stride[0] % 8 ||
+      out->stride[1] % 8)
+    return fail(PA_ERR_INVALID_ARG, "q/out rows must be 16-byte aligned");
+  if (!aligned(k_cache->data, 128) || !aligned(v_cache->data, 128))
+    return fail(PA_ERR_INVALID_ARG, "caches must be 128-byte aligned");
+  if (block_tables->stride[1] != 1 && block_tables->shape[1] > 1)
+    return fail(PA_ERR_INVALID_ARG, "block_tables last stride must be 1");
+  if (context_lens->stride[0] != 1 && B > 1) return fail(PA_ERR_INVALID_ARG, "context_lens must be contiguous");
+  if (!out->data || !q->data || !k_cache->data || !v_cache->data || !block_tables->data || !context_lens->data)
+    return fail(PA_ERR_INVALID_ARG, "NULL data pointer");
+  const int64_t max_blocks = block_tables->shape[1];
+  if (max_blocks <= 0) return fail(PA_ERR_INVALID_ARG, "block_tables has no columns");
+
+  pa::DecodeConfig cfg{};
+  cfg.kv = cd == PA_E4M3 ? pa::KvType::E4M3 : (cd == PA_BF16 ? pa::KvType::BF16 : pa::KvType::F16);
+  cfg.q = q->dtype == PA_BF16 ? pa::QType::BF16 : pa::QType::F16;
+  cfg.head_dim = static_cast<int>(D);
+  cfg.ntiles = static_cast<int>((G + 7) / 8);
+  cfg.kernel = opts.kernel < 0 ? 1 : opts.kernel;
+  if (cfg.kernel != 0 && cfg.kernel != 1) return fail(PA_ERR_INVALID_ARG, "opts.kernel must be -1, 0 or 1");
+  if (!pa::decode_supported(cfg))
+    return fail(PA_ERR_UNSUPPORTED, "no kernel for head_dim %lld, cache %s, q %s, group %lld, kernel %d", (long long)D,
+                dtype_name(cd), dtype_name(q->dtype), (long long)G, cfg.kernel);
+
+  float k_scale = 1.f, v_scale = 1.f;
+  if (cd == PA_E4M3) {
+    k_scale = opts.k_scale;
+    v_scale = opts.v_scale;
+    if (!(std::isfinite(k_scale) && k_scale > 0.f && std::isfinite(v_scale) && v_scale > 0.f))
+      return fail(PA_ERR_INVALID_ARG, "E4M3 cache scales must be finite and > 0");
+  }
+
+  int64_t max_ctx = opts.max_context_len > 0 ? opts.max_context_len : max_blocks * 16;
+  if (opts.max_context_len < 0) return fail(PA_ERR_INVALID_ARG, "max_context_len < 0");
+  max_ctx = std::min<int64_t>(max_ctx, max_blocks * 16);
+  int64_t pt = opts.partition_tokens;
+  if (pt < 0 || pt % 16 || pt > pa::kMaxPartitionTokens)
+    return fail(PA_ERR_INVALID_ARG, "partition_tokens %lld must be a multiple of 16 in [0, %d]", (long long)pt,
+                pa::kMaxPartitionTokens);
+  const bool have_ws = opts.workspace != nullptr && opts.workspace_bytes > 0;
+  if (pt == 0) {
+    pt = auto_partition_tokens(static_cast<int32_t>(max_ctx));
+    if (pt == 0 || (!have_ws && max_ctx <= pa::kMaxPartitionTokens)) pt = std::max<int64_t>(16, (max_ctx + 15) / 16 * 16);
+  }
+  int64_t P = (max_ctx + pt - 1) / pt;
+  if (P < 1) P = 1;
+  if (P > 0x7fffffff) return fail(PA_ERR_UNSUPPORTED, "too many partitions");
+
+  pa::DecodeParams p{};
+  p.out = out->data;
+  p.q = q->data;
+  p.q_stride_s = q->stride[0];
+  p.q_stride_h = q->stride[1];
+  p.o_stride_s = out->stride[0];
+  p.o_stride_h = out->stride[1];
+  p.block_tables = static_cast<const int32_t*>(block_tables->data);
+  p.bt_stride = block_tables->stride[0];
+  p.context_lens = static_cast<const int32_t*>(context_lens->data);
+  p.num_seqs = static_cast<int32_t>(B);
+  p.num_blocks = static_cast<int32_t>(NB);
+  p.num_kv_heads = num_kv_heads;
+  p.group = static_cast<int32_t>(G);
+  p.max_blocks = static_cast<int32_t>(std::min<int64_t>(max_blocks, 0x7fffffff / 16));
+  p.partition_tokens = static_cast<int32_t>(pt);
+  p.num_partitions = static_cast<int32_t>(P);
+  p.score_scale_log2 = scale * 1.4426950408889634f * k_scale;
+  p.v_scale = v_scale;
+  p.err = opts.error_word ? reinterpret_cast<uint32_t*>(opts.error_word) : library_error_word();
+  if (!p.err) return fail(PA_ERR_CUDA, "no device error word (no current CUDA device?)");
+  if (P > 1) {
+    size_t ml_off = 0;
+    const size_t need = workspace_layout(B, Hq, D, P, &ml_off);
+    if (!have_ws || opts.workspace_bytes < need)
+      return fail(PA_ERR_WORKSPACE, "split into %lld partitions needs a workspace of %zu bytes (got %zu)", (long long)P,
+                  need, have_ws ? opts.workspace_bytes : size_t(0));
+    if (!aligned(opts.workspace, 256)) return fail(PA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    p.ws_acc = static_cast<float*>(opts.workspace);
+    p.ws_ml = reinterpret_cast<float*>(static_cast<char*>(opts.workspace) + ml_off);
+  }
+
+  CUtensorMap km, vm;
+  const int esz = elem_bytes(cd);
+  if ((st = encode_pool_map(&km, k_cache, esz)) || (st = encode_pool_map(&vm, v_cache, esz))) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = pa::launch_decode(cfg, km, vm, p, s);
+  if (e != cudaSuccess) return fail(PA_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
+  if (P > 1) {
+    e = pa::launch_reduce(cfg, p, s);
+    if (e != cudaSuccess) return fail(PA_ERR_CUDA, "reduce launch: %s", cudaGetErrorString(e));
+  }
+  return ok();
+}
+
+}  // extern "C"

@@ -1,0 +1,75 @@
+// Internal launch interface between the C-ABI layer (api.cu) and the kernel translation units.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace pa {
+
+enum class KvType : int { F16 = 0, BF16 = 1, E4M3 = 2 };
+enum class QType : int { F16 = 0, BF16 = 1 };
+
+// Kernel-side view of one pa_decode call. Strides are in elements.
+struct DecodeParams {
+  void* out;
+  const void* q;
+  int64_t q_stride_s, q_stride_h;
+  int64_t o_stride_s, o_stride_h;
+  const int32_t* block_tables;
+  int64_t bt_stride;
+  const int32_t* context_lens;
+  int32_t num_seqs;
+  int32_t num_blocks;
+  int32_t num_kv_heads;
+  int32_t group;             // query heads per KV head
+  int32_t max_blocks;        // block-table width
+  int32_t partition_tokens;  // tokens per partition (multiple of 16)
+  int32_t num_partitions;    // grid.x; 1 = no split (decode writes out directly)
+  float score_scale_log2;    // scale * log2(e) * k_scale (e4m3) -- folded into the scores
+  float v_scale;             // applied once to the normalised output (e4m3), 1 otherwise
+  float* ws_acc;             // [B, Hq, P, D] un-normalised partial outputs (split only)
+  float* ws_ml;              // [B, Hq, P, 2] partial (running max in log2 units, sum) (split only)
+  uint32_t* err;             // error word (never null)
+};
+
+struct DecodeConfig {
+  KvType kv;
+  QType q;
+  int head_dim;  // 64 or 128
+  int ntiles;    // ceil(group / 8): 1 or 2
+  int kernel;    // 0 = CUDA-core FMA, 1 = tensor-core mma.sync
+};
+
+// Number of warps per CTA of the decode kernels; a partition holds at most 32 pages per warp.
+constexpr int kDecodeWarps = 4;
+constexpr int kMaxPartitionTokens = 16 * 32 * kDecodeWarps;
+
+cudaError_t launch_decode(const DecodeConfig& cfg, const CUtensorMap& k_map, const CUtensorMap& v_map,
+                          const DecodeParams& p, cudaStream_t stream);
+cudaError_t launch_reduce(const DecodeConfig& cfg, const DecodeParams& p, cudaStream_t stream);
+bool decode_supported(const DecodeConfig& cfg);
+
+struct CacheParams {
+  const void* key;
+  const void* value;
+  int64_t k_stride_t, k_stride_h;
+  int64_t v_stride_t, v_stride_h;
+  const int64_t* slots;
+  void* k_cache;
+  void* v_cache;
+  int64_t num_tokens;
+  int32_t num_kv_heads;
+  int32_t head_dim;
+  int64_t num_slots;  // num_blocks * 16
+  float k_inv_scale, v_inv_scale;
+  uint32_t* err;
+};
+
+// src: 0 = f16, 1 = bf16 source; cache: KvType.
+cudaError_t launch_reshape_and_cache(int src_bf16, KvType cache, const CacheParams& p, cudaStream_t stream);
+
+uint32_t* decode_error_word();  // device address of the library's own error word
+cudaError_t read_and_clear_error_word(uint32_t* bits, int clear);
+
+}  // namespace pa

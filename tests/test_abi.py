@@ -1,0 +1,135 @@
+"""CPU checks of the C-ABI library: it loads, exports every declared entry point, and its host-side
+allocator and slot helper agree with the oracle's models. No GPU and no device compute here."""
+import ctypes
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+import torch
+from hypothesis import given, settings
+from hypothesis import strategies as st
+
+import paged_kv_cache_385_b200 as pa
+import workloads as W
+from oracle import paging
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    names = []
+    for hdr in os.listdir(os.path.join(ROOT, "include")):
+        if not hdr.endswith(".h"):
+            continue
+        text = open(os.path.join(ROOT, "include", hdr)).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names += re.findall(r"\b(pa_[a-z0-9_]+)\s*\(", text)
+    return sorted(set(names))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("pa_reshape_and_cache", "pa_decode", "pa_decode_workspace_bytes", "pa_allocator_create",
+                     "pa_block_alloc", "pa_block_incref", "pa_block_free", "pa_status_string"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(pa.LIB_PATH)
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+    out = subprocess.run(["nm", "-D", "--defined-only", pa.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r" T (pa_[a-z0-9_]+)$", out, flags=re.M))
+    assert set(declared_functions()) <= exported
+
+
+def test_status_strings_and_version():
+    assert pa.pa_status_string(pa.PA_OK) == "ok"
+    assert pa.pa_status_string(pa.PA_ERR_WORKSPACE).startswith("workspace")
+    assert re.match(r"^\d+\.\d+\.\d+$", pa.pa_version())
+
+
+def test_workspace_sizing():
+    assert pa.pa_decode_workspace_bytes(4, 4, 64, 100, 0) == 0  # fits one partition
+    assert pa.pa_decode_partition_tokens(8, 8, 131072) == 512
+    n = pa.pa_decode_workspace_bytes(8, 64, 128, 131072, 512)
+    P = 131072 // 512
+    assert n >= 8 * 64 * P * (128 + 2) * 4
+
+
+def test_null_tensor_is_rejected_without_a_gpu():
+    lib = pa.lib()
+    st_ = lib.pa_decode(None, None, None, None, None, None, 1.0, 1, None, None)
+    assert st_ == pa.PA_ERR_INVALID_ARG
+    assert "NULL" in pa.pa_last_error()
+
+
+@settings(max_examples=150, deadline=None)
+@given(n=st.integers(1, 40), ops=st.lists(st.tuples(st.sampled_from("aif"), st.integers(-2, 42)), max_size=150),
+       seed=st.integers(0, 2**31 - 1))
+def test_allocator_matches_oracle_model(n, ops, seed):
+    order = np.random.default_rng(seed).permutation(n).tolist()
+    model = paging.FreeListModel(n, order)
+    a = pa.BlockAllocator(n, order)
+    lib = pa.lib()
+    for op, b in ops:
+        if op == "a":
+            want = model.alloc()
+            got = lib.pa_block_alloc(a._h)
+            assert got == (pa.PA_ERR_EXHAUSTED if want is None else want)
+        elif op == "i":
+            assert (lib.pa_block_incref(a._h, b) == pa.PA_OK) == model.incref(b)
+        else:
+            assert (lib.pa_block_free(a._h, b) == pa.PA_OK) == model.free(b)
+        assert a.num_free == model.num_free
+    for blk in range(n):
+        assert a.refcount(blk) == model.refcount(blk)
+    assert lib.pa_block_refcount(a._h, n) == pa.PA_ERR_BAD_BLOCK
+
+
+def test_allocator_rejects_bad_orders():
+    with pytest.raises(ValueError):
+        pa.BlockAllocator(4, [0, 1, 1, 2])
+    with pytest.raises(ValueError):
+        pa.BlockAllocator(4, [0, 1, 2, 4])
+    with pytest.raises(ValueError):
+        pa.BlockAllocator(0)
+
+
+def test_alloc_n_is_all_or_nothing():
+    a = pa.BlockAllocator(5)
+    a.alloc_n(3)
+    with pytest.raises(pa.PagedAttentionError) as e:
+        a.alloc_n(3)
+    assert e.value.status == pa.PA_ERR_EXHAUSTED
+    assert a.num_free == 2
+
+
+@pytest.mark.parametrize("name", ["tiny", "llama3_8b_gqa_small", "prefix_gqa_small", "long70b_fp8_small",
+                                  "llama3_8b_gqa", "prefix_gqa", "long70b_fp8"])
+def test_block_tables_and_slots_match_oracle(name):
+    w = W.ALL[name]
+    lens = W.context_lens(w)
+    order = W.block_order(w)
+    mb = W.max_blocks_per_seq(w, lens)
+    bt = pa.build_block_tables(pa.BlockAllocator(w.num_blocks, order.tolist()), lens.tolist(), mb,
+                               w.shared_prefix_tokens)
+    bt_o = paging.build_block_tables(lens.numpy(), order.numpy(), w.num_blocks, 16, w.shared_prefix_tokens, mb)
+    assert np.array_equal(bt.numpy(), bt_o)
+    rng = np.random.default_rng(3)
+    seqs = rng.integers(0, w.num_seqs, 200)
+    poss = [int(rng.integers(0, int(lens[s]))) for s in seqs]
+    got = pa.pa_slots_for_positions(bt, seqs.tolist(), poss).numpy()
+    want = paging.slots_for_positions(bt_o, seqs.tolist(), poss)
+    assert np.array_equal(got, want)
+
+
+def test_slot_helper_rejects_out_of_range():
+    bt = torch.tensor([[3, -1]], dtype=torch.int32)
+    with pytest.raises(pa.PagedAttentionError):
+        pa.pa_slots_for_positions(bt, [0], [16])  # entry -1
+    with pytest.raises(pa.PagedAttentionError):
+        pa.pa_slots_for_positions(bt, [0], [40])  # beyond the table
+    assert pa.pa_slots_for_positions(bt, [0], [5]).tolist() == [53]
