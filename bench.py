@@ -169,7 +169,7 @@ class Setup:
         self.lens = lens.to(device)
         pt = w.partition_tokens if partition_tokens is None else partition_tokens
         self.pt = pt
-        self.ws = pa.decode_workspace(B, w.num_q_heads, w.head_dim, self.max_ctx, pt, device=device)
+        self.ws = pa.decode_workspace(B, w.num_q_heads, w.num_kv_heads, w.head_dim, self.max_ctx, pt, device=device)
         self.opts = pa.decode_opts(k_scale=self.k_scale, v_scale=self.v_scale, max_context_len=self.max_ctx,
                                    partition_tokens=pt, workspace=self.ws, kernel=kernel)
         eff_pt = pt if pt else pa.pa_decode_partition_tokens(B, w.num_kv_heads, self.max_ctx)

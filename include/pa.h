@@ -140,12 +140,14 @@ int pa_decode(pa_tensor* out, const pa_tensor* q, const pa_tensor* k_cache, cons
               const pa_decode_opts* opts, void* stream);
 
 /* Partition size pa_decode uses when opts->partition_tokens == 0 and a workspace is given
- * (0 = no split). Host only. */
+ * (0 = no split: the batch's B * Hkv (sequence, KV head) units already fill the GPU and every
+ * context fits one CTA, <= 2048 tokens). Otherwise the largest of 2048, 1024, 512 that still gives
+ * about four CTAs per SM, else 256. Host only. */
 int32_t pa_decode_partition_tokens(int32_t num_seqs, int32_t num_kv_heads, int32_t max_context_len);
 
 /* Workspace bytes pa_decode needs for these sizes (0 when no split happens). partition_tokens 0
- * applies the library's choice. Host only. */
-size_t pa_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t head_dim,
+ * applies pa_decode_partition_tokens. Host only. */
+size_t pa_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
                                  int32_t max_context_len, int32_t partition_tokens);
 
 /* Static string for a pa_status value. */

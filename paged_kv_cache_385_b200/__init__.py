@@ -17,7 +17,8 @@ from typing import Optional, Sequence
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libpagedattn.so")
+# PAGED_KV_CACHE_LIB points the binding at another build of the library (e.g. a tuning variant).
+LIB_PATH = os.environ.get("PAGED_KV_CACHE_LIB") or os.path.join(_HERE, "libpagedattn.so")
 
 PA_OK = 0
 PA_ERR_INVALID_ARG = -1
@@ -76,7 +77,7 @@ def _load() -> ctypes.CDLL:
         "pa_reshape_and_cache": (ctypes.c_int, [P, P, P, P, P, F32, F32, VP]),
         "pa_decode": (ctypes.c_int, [P, P, P, P, P, P, F32, I32, ctypes.POINTER(PaDecodeOpts), VP]),
         "pa_decode_partition_tokens": (I32, [I32, I32, I32]),
-        "pa_decode_workspace_bytes": (SZ, [I32, I32, I32, I32, I32]),
+        "pa_decode_workspace_bytes": (SZ, [I32, I32, I32, I32, I32, I32]),
         "pa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         "pa_last_error": (ctypes.c_char_p, []),
         "pa_read_device_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), ctypes.c_int]),
@@ -197,15 +198,16 @@ def pa_decode_partition_tokens(num_seqs: int, num_kv_heads: int, max_context_len
     return int(_lib.pa_decode_partition_tokens(num_seqs, num_kv_heads, max_context_len))
 
 
-def pa_decode_workspace_bytes(num_seqs: int, num_q_heads: int, head_dim: int, max_context_len: int,
-                              partition_tokens: int = 0) -> int:
-    return int(_lib.pa_decode_workspace_bytes(num_seqs, num_q_heads, head_dim, max_context_len, partition_tokens))
+def pa_decode_workspace_bytes(num_seqs: int, num_q_heads: int, num_kv_heads: int, head_dim: int,
+                              max_context_len: int, partition_tokens: int = 0) -> int:
+    return int(_lib.pa_decode_workspace_bytes(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len,
+                                              partition_tokens))
 
 
-def decode_workspace(num_seqs: int, num_q_heads: int, head_dim: int, max_context_len: int, partition_tokens: int = 0,
-                     device=None) -> Optional[torch.Tensor]:
+def decode_workspace(num_seqs: int, num_q_heads: int, num_kv_heads: int, head_dim: int, max_context_len: int,
+                     partition_tokens: int = 0, device=None) -> Optional[torch.Tensor]:
     """A device workspace big enough for these sizes (None when no split happens)."""
-    n = pa_decode_workspace_bytes(num_seqs, num_q_heads, head_dim, max_context_len, partition_tokens)
+    n = pa_decode_workspace_bytes(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len, partition_tokens)
     if n == 0:
         return None
     return torch.empty(n, dtype=torch.uint8, device=device or "cuda")

@@ -125,7 +125,18 @@ uint32_t* library_error_word() {
   return words[dev];
 }
 
-int32_t auto_partition_tokens(int32_t max_ctx) { return max_ctx > 512 ? 512 : 0; }
+// Split only when the batch alone cannot fill the GPU: with B * Hkv work units of up to 2048 tokens
+// there are enough CTAs once B * Hkv >= kFillUnits; otherwise take the largest partition (fewer,
+// longer CTAs: less prologue and merge work) that still yields kFillUnits CTAs.
+constexpr int64_t kFillUnits = 4 * 148;
+
+int32_t auto_partition_tokens(int32_t num_seqs, int32_t num_kv_heads, int32_t max_ctx) {
+  const int64_t units = static_cast<int64_t>(num_seqs) * num_kv_heads;
+  if (max_ctx <= pa::kMaxPartitionTokens && units >= kFillUnits) return 0;
+  for (int32_t pt = pa::kMaxPartitionTokens; pt > 256; pt /= 2)
+    if (units * ((max_ctx + pt - 1) / pt) >= kFillUnits && max_ctx > pt) return pt;
+  return max_ctx > 256 ? 256 : 0;
+}
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -167,15 +178,15 @@ void pa_decode_opts_init(pa_decode_opts* o) {
 }
 
 int32_t pa_decode_partition_tokens(int32_t num_seqs, int32_t num_kv_heads, int32_t max_context_len) {
-  (void)num_seqs;
-  (void)num_kv_heads;
-  return auto_partition_tokens(max_context_len);
+  if (num_seqs <= 0 || num_kv_heads <= 0 || max_context_len <= 0) return 0;
+  return auto_partition_tokens(num_seqs, num_kv_heads, max_context_len);
 }
 
-size_t pa_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t head_dim, int32_t max_context_len,
-                                 int32_t partition_tokens) {
-  if (num_seqs <= 0 || num_q_heads <= 0 || head_dim <= 0 || max_context_len <= 0) return 0;
-  const int32_t pt = partition_tokens > 0 ? partition_tokens : auto_partition_tokens(max_context_len);
+size_t pa_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                 int32_t max_context_len, int32_t partition_tokens) {
+  if (num_seqs <= 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || max_context_len <= 0) return 0;
+  const int32_t pt =
+      partition_tokens > 0 ? partition_tokens : auto_partition_tokens(num_seqs, num_kv_heads, max_context_len);
   if (pt <= 0) return 0;
   const int64_t P = (static_cast<int64_t>(max_context_len) + pt - 1) / pt;
   if (P <= 1) return 0;
@@ -345,7 +356,7 @@ int pa_decode(pa_tensor* out, const pa_tensor* q, const pa_tensor* k_cache, cons
                 pa::kMaxPartitionTokens);
   const bool have_ws = opts.workspace != nullptr && opts.workspace_bytes > 0;
   if (pt == 0) {
-    pt = auto_partition_tokens(static_cast<int32_t>(max_ctx));
+    pt = auto_partition_tokens(static_cast<int32_t>(B), num_kv_heads, static_cast<int32_t>(max_ctx));
     if (pt == 0 || (!have_ws && max_ctx <= pa::kMaxPartitionTokens)) pt = std::max<int64_t>(16, (max_ctx + 15) / 16 * 16);
   }
   int64_t P = (max_ctx + pt - 1) / pt;

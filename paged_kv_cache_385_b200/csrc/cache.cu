@@ -5,9 +5,13 @@
 // [Hkv, D] goes to k_cache[slot / 16, :, slot % 16, :] (V likewise). A 16-bit cache stores the
 // bits unchanged; an e4m3 cache stores e4m3_rn_satfinite(float32(x) * float32(1 / scale)).
 //
-// One CTA per token; each thread moves 16-byte chunks (8 elements) of the token's K and V rows
-// for all heads: 16-byte loads from the [T, Hkv, D] inputs, 16-byte (or 8-byte for e4m3) stores
-// into the pool. Slot -1 skips the token; a slot outside the pool is skipped and reported.
+// Grid (tokens, chunk groups): each thread moves one 16-byte chunk (8 elements) of a token's K or V
+// row, so every load of a token is in flight at once (the step writes only a few hundred KB, so
+// latency, not bandwidth, sets its time): a 16-byte load from the [T, Hkv, D] input, a 16-byte (or
+// 8-byte for e4m3) store into the pool. Slot -1 skips the token; a slot outside the pool is
+// skipped and reported.
+#include <algorithm>
+
 #include "internal.h"
 #include "pa_device.cuh"
 
@@ -20,14 +24,14 @@ __global__ void __launch_bounds__(128) reshape_and_cache_kernel(const CacheParam
   const int64_t slot = p.slots[t];
   if (slot == -1) return;
   if (slot < -1 || slot >= p.num_slots) {
-    if (threadIdx.x == 0) atomicOr(p.err, 2u);
+    if (threadIdx.x == 0 && blockIdx.y == 0) atomicOr(p.err, 2u);
     return;
   }
   const int64_t blk = slot >> 4, off = slot & 15;
   const int D = p.head_dim;
   const int chunks_per_head = D / 8;
   const int nchunks = p.num_kv_heads * chunks_per_head;
-  for (int c = threadIdx.x; c < 2 * nchunks; c += blockDim.x) {
+  for (int c = blockIdx.y * blockDim.x + threadIdx.x; c < 2 * nchunks; c += gridDim.y * blockDim.x) {
     const bool is_v = c >= nchunks;
     const int cc = is_v ? c - nchunks : c;
     const int h = cc / chunks_per_head, d0 = (cc % chunks_per_head) * 8;
@@ -58,7 +62,9 @@ __global__ void __launch_bounds__(128) reshape_and_cache_kernel(const CacheParam
 
 cudaError_t launch_reshape_and_cache(int src_bf16, KvType cache, const CacheParams& p, cudaStream_t st) {
   if (p.num_tokens == 0) return cudaSuccess;
-  const dim3 grid(static_cast<unsigned>(p.num_tokens));
+  const int chunks = 2 * p.num_kv_heads * (p.head_dim / 8);
+  const unsigned groups = static_cast<unsigned>(std::min(65535, (chunks + 127) / 128));
+  const dim3 grid(static_cast<unsigned>(p.num_tokens), groups);
   if (cache == KvType::E4M3) {
     if (src_bf16) reshape_and_cache_kernel<true, KvType::E4M3><<<grid, 128, 0, st>>>(p);
     else reshape_and_cache_kernel<false, KvType::E4M3><<<grid, 128, 0, st>>>(p);

@@ -36,6 +36,22 @@ namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;
 
+// Shared-memory budget of a CTA's page pipeline, and the CTAs per SM the kernel is compiled for.
+// 16-bit pages are bandwidth-bound (deep pipelines, 2 CTAs/SM); e4m3 pages carry 3x the math per
+// byte, so they trade stages for more resident warps.
+#ifndef PA_PIPE_BYTES_16
+#define PA_PIPE_BYTES_16 (96 * 1024)
+#endif
+#ifndef PA_MIN_BLOCKS_16
+#define PA_MIN_BLOCKS_16 2
+#endif
+#ifndef PA_PIPE_BYTES_8
+#define PA_PIPE_BYTES_8 (96 * 1024)
+#endif
+#ifndef PA_MIN_BLOCKS_8
+#define PA_MIN_BLOCKS_8 2
+#endif
+
 template <KvType KV, QType QT, int D, int NT, int KIND>
 struct Cfg {
   static constexpr bool kFp8 = KV == KvType::E4M3;
@@ -47,7 +63,9 @@ struct Cfg {
   static constexpr int kWarps = kDecodeWarps;
   static constexpr int kThreads = kWarps * 32;
   static constexpr int kStageBytes = 2 * kPageBytes;  // K page + V page
-  static constexpr int kStages = (96 * 1024) / (kWarps * kStageBytes);
+  static constexpr int kPipeBudget = kFp8 ? PA_PIPE_BYTES_8 : PA_PIPE_BYTES_16;
+  static constexpr int kMinBlocks = kFp8 ? PA_MIN_BLOCKS_8 : PA_MIN_BLOCKS_16;
+  static constexpr int kStages = kPipeBudget / (kWarps * kStageBytes);
   static constexpr int kPipeBytes = kWarps * kStages * kStageBytes;
   static constexpr bool kMmaBf16 = KV == KvType::BF16;  // e4m3 pages are widened to f16
   static constexpr bool kQBf16 = QT == QType::BF16;
@@ -437,7 +455,7 @@ struct FmaMath {
 // The decode kernel: pipeline, per-warp loop, merge, epilogue.
 // ---------------------------------------------------------------------------------------------
 template <KvType KV, QType QT, int D, int NT, int KIND>
-__global__ void __launch_bounds__(Cfg<KV, QT, D, NT, KIND>::kThreads, 2)
+__global__ void __launch_bounds__(Cfg<KV, QT, D, NT, KIND>::kThreads, Cfg<KV, QT, D, NT, KIND>::kMinBlocks)
     decode_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
                   const DecodeParams p) {
   using C = Cfg<KV, QT, D, NT, KIND>;
@@ -683,7 +701,9 @@ cudaError_t launch_one(const CUtensorMap& km, const CUtensorMap& vm, const Decod
 template <KvType KV, QType QT, int D, int KIND>
 cudaError_t launch_nt(int nt, const CUtensorMap& km, const CUtensorMap& vm, const DecodeParams& p, cudaStream_t st) {
   if (nt == 1) return launch_one<KV, QT, D, 1, KIND>(km, vm, p, st);
-  if (KIND == 1 && nt == 2) return launch_one<KV, QT, D, 2, KIND>(km, vm, p, st);
+  if constexpr (KIND == 1) {
+    if (nt == 2) return launch_one<KV, QT, D, 2, KIND>(km, vm, p, st);
+  }
   return cudaErrorInvalidValue;
 }
 

@@ -96,7 +96,7 @@ class DeviceCase:
 
     def workspace(self, partition_tokens: int = 0) -> Optional[torch.Tensor]:
         w = self.w
-        return pa.decode_workspace(w.num_seqs, w.num_q_heads, w.head_dim, self.max_ctx, partition_tokens)
+        return pa.decode_workspace(w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim, self.max_ctx, partition_tokens)
 
     def decode(self, kernel: int = -1, partition_tokens: Optional[int] = None, out: Optional[torch.Tensor] = None,
                error_word: Optional[torch.Tensor] = None) -> torch.Tensor:

@@ -52,9 +52,13 @@ def test_status_strings_and_version():
 
 
 def test_workspace_sizing():
-    assert pa.pa_decode_workspace_bytes(4, 4, 64, 100, 0) == 0  # fits one partition
-    assert pa.pa_decode_partition_tokens(8, 8, 131072) == 512
-    n = pa.pa_decode_workspace_bytes(8, 64, 128, 131072, 512)
+    assert pa.pa_decode_workspace_bytes(4, 4, 4, 64, 100, 0) == 0  # fits one partition
+    assert pa.pa_decode_partition_tokens(32, 32, 2048) == 0  # 1024 units fill the GPU unsplit
+    assert pa.pa_decode_partition_tokens(8, 8, 131072) == 2048
+    assert pa.pa_decode_partition_tokens(64, 8, 8192) == 2048
+    assert pa.pa_decode_partition_tokens(1, 8, 32768) == 256
+    assert pa.pa_decode_partition_tokens(4, 8, 4096) == 256
+    n = pa.pa_decode_workspace_bytes(8, 64, 8, 128, 131072, 512)
     P = 131072 // 512
     assert n >= 8 * 64 * P * (128 + 2) * 4
 
