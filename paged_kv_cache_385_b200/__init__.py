@@ -5,7 +5,7 @@ become ``pa_tensor`` views, the current CUDA stream is passed through, a non-OK 
 ``PagedAttentionError``. Every step of the hot path runs in the library's CUDA kernels; there is no
 CPU fallback. Device arguments must be CUDA tensors.
 
-Build the library first (``python -m paged_kv_cache_385_b200.build``); importing this package
+Build the library first (``python paged_kv_cache_385_b200/build.py``); importing this package
 without it raises ImportError.
 """
 from __future__ import annotations
@@ -67,7 +67,7 @@ class PagedAttentionError(RuntimeError):
 
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"{LIB_PATH} is not built; run `python -m paged_kv_cache_385_b200.build`")
+        raise ImportError(f"{LIB_PATH} is not built; run `python paged_kv_cache_385_b200/build.py`")
     lib = ctypes.CDLL(LIB_PATH)
     P, I32, I64, F32, SZ, VP = (ctypes.POINTER(PaTensor), ctypes.c_int32, ctypes.c_int64, ctypes.c_float,
                                 ctypes.c_size_t, ctypes.c_void_p)

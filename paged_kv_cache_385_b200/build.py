@@ -1,6 +1,9 @@
 """Build libpagedattn.so in-tree with nvcc for sm_100a (no GPU needed: nvcc cross-compiles).
 
-    python -m paged_kv_cache_385_b200.build [--force] [--verbose]
+    python paged_kv_cache_385_b200/build.py [--force] [--verbose] [--ptxas-v]
+
+Run it as a file, not as ``-m paged_kv_cache_385_b200.build``: importing the package loads the
+library, which is what this script produces.
 
 Objects go to ``<package>/_build``; the shared library to ``<package>/libpagedattn.so``.
 A rebuild happens when any source or header is newer than the library.

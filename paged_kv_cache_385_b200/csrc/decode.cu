@@ -36,23 +36,12 @@ namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;
 
-// Shared-memory budget of a CTA's page pipeline, and the CTAs per SM the kernel is compiled for.
-// 16-bit pages are bandwidth-bound (deep pipelines, 2 CTAs/SM); e4m3 pages carry 3x the math per
-// byte, so they trade stages for more resident warps.
-#ifndef PA_PIPE_BYTES_16
-#define PA_PIPE_BYTES_16 (96 * 1024)
-#endif
-#ifndef PA_MIN_BLOCKS_16
-#define PA_MIN_BLOCKS_16 2
-#endif
-#ifndef PA_PIPE_BYTES_8
-#define PA_PIPE_BYTES_8 (96 * 1024)
-#endif
-#ifndef PA_MIN_BLOCKS_8
-#define PA_MIN_BLOCKS_8 2
-#endif
-
-template <KvType KV, QType QT, int D, int NT, int KIND>
+// OCC is the number of CTAs per SM a kernel is compiled for: the page pipeline gets 192 KB / OCC of
+// shared memory (96, 64 or 48 KB) and registers are capped to fit. 16-bit pages with one query per
+// KV head are pure bandwidth: deep pipelines, 2 CTAs/SM. Grouped queries add math per byte and
+// e4m3 pages even more (widening, 3x the pages per byte moved), so those trade stages for resident
+// warps: 3 and 4 CTAs/SM.
+template <KvType KV, QType QT, int D, int NT, int KIND, int OCC>
 struct Cfg {
   static constexpr bool kFp8 = KV == KvType::E4M3;
   static constexpr int kEsz = kFp8 ? 1 : 2;
@@ -63,8 +52,8 @@ struct Cfg {
   static constexpr int kWarps = kDecodeWarps;
   static constexpr int kThreads = kWarps * 32;
   static constexpr int kStageBytes = 2 * kPageBytes;  // K page + V page
-  static constexpr int kPipeBudget = kFp8 ? PA_PIPE_BYTES_8 : PA_PIPE_BYTES_16;
-  static constexpr int kMinBlocks = kFp8 ? PA_MIN_BLOCKS_8 : PA_MIN_BLOCKS_16;
+  static constexpr int kMinBlocks = OCC;
+  static constexpr int kPipeBudget = OCC == 2 ? 96 * 1024 : (OCC == 3 ? 64 * 1024 : 48 * 1024);
   static constexpr int kStages = kPipeBudget / (kWarps * kStageBytes);
   static constexpr int kPipeBytes = kWarps * kStages * kStageBytes;
   static constexpr bool kMmaBf16 = KV == KvType::BF16;  // e4m3 pages are widened to f16
@@ -157,10 +146,12 @@ struct TcMath {
       for (int kp = 0; kp < KS / 2; ++kp) {
         uint32_t raw[4];
         ldmatrix_x4(raw, kb + swz(a_tok, 2 * kp + a_co));
-        uint32_t a0[4] = {e4m3x2_to_f16x2(raw[0]), e4m3x2_to_f16x2(raw[1]), e4m3x2_to_f16x2(raw[0] >> 16),
-                          e4m3x2_to_f16x2(raw[1] >> 16)};
-        uint32_t a1[4] = {e4m3x2_to_f16x2(raw[2]), e4m3x2_to_f16x2(raw[3]), e4m3x2_to_f16x2(raw[2] >> 16),
-                          e4m3x2_to_f16x2(raw[3] >> 16)};
+        // a0a1 / a2a3 take codes (d 4q, 4q+1) of tokens r / r+8; a4a5 / a6a7 take (d 4q+2, 4q+3).
+        uint32_t a0[4], a1[4];
+        e4m3x4_to_f16x2x2(raw[0], a0[0], a0[2]);
+        e4m3x4_to_f16x2x2(raw[1], a0[1], a0[3]);
+        e4m3x4_to_f16x2x2(raw[2], a1[0], a1[2]);
+        e4m3x4_to_f16x2x2(raw[3], a1[1], a1[3]);
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
           mma_16816<false>(sc[nt], a0, qf[nt][2 * kp][0], qf[nt][2 * kp][1]);
@@ -229,10 +220,16 @@ struct TcMath {
         ldmatrix_x4_trans(raw, vb + swz(a_tok, 2 * mp + a_co));
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
+          // (tok 2q, d), (tok 2q, d+1), (tok 2q+1, d), (tok 2q+1, d+1) -> pairs of tokens per d.
           const uint32_t t0 = __byte_perm(raw[2 * half], 0, 0x3120);
           const uint32_t t1 = __byte_perm(raw[2 * half + 1], 0, 0x3120);
-          uint32_t a[4] = {e4m3x2_to_f16x2(t0) & mlo, e4m3x2_to_f16x2(t0 >> 16) & mlo,
-                           e4m3x2_to_f16x2(t1) & mhi, e4m3x2_to_f16x2(t1 >> 16) & mhi};
+          uint32_t a[4];
+          e4m3x4_to_f16x2x2(t0, a[0], a[1]);
+          e4m3x4_to_f16x2x2(t1, a[2], a[3]);
+          a[0] &= mlo;
+          a[1] &= mlo;
+          a[2] &= mhi;
+          a[3] &= mhi;
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt) mma_16816<false>(acc[nt][2 * mp + half], a, pf[nt][0], pf[nt][1]);
         }
@@ -331,8 +328,9 @@ struct FmaMath {
   }
 
   __device__ __forceinline__ static void widen8(uint32_t lo, uint32_t hi, float (&f)[8]) {
-    const uint32_t w[4] = {e4m3x2_to_f16x2(lo), e4m3x2_to_f16x2(lo >> 16), e4m3x2_to_f16x2(hi),
-                           e4m3x2_to_f16x2(hi >> 16)};
+    uint32_t w[4];
+    e4m3x4_to_f16x2x2(lo, w[0], w[1]);
+    e4m3x4_to_f16x2x2(hi, w[2], w[3]);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const float2 t = unpack2<false>(w[i]);
@@ -454,11 +452,11 @@ struct FmaMath {
 // ---------------------------------------------------------------------------------------------
 // The decode kernel: pipeline, per-warp loop, merge, epilogue.
 // ---------------------------------------------------------------------------------------------
-template <KvType KV, QType QT, int D, int NT, int KIND>
-__global__ void __launch_bounds__(Cfg<KV, QT, D, NT, KIND>::kThreads, Cfg<KV, QT, D, NT, KIND>::kMinBlocks)
+template <KvType KV, QType QT, int D, int NT, int KIND, int OCC>
+__global__ void __launch_bounds__(Cfg<KV, QT, D, NT, KIND, OCC>::kThreads, Cfg<KV, QT, D, NT, KIND, OCC>::kMinBlocks)
     decode_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
                   const DecodeParams p) {
-  using C = Cfg<KV, QT, D, NT, KIND>;
+  using C = Cfg<KV, QT, D, NT, KIND, OCC>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kPipeBytes);
@@ -677,41 +675,47 @@ __global__ void __launch_bounds__(D) reduce_kernel(const DecodeParams p) {
   static_cast<uint16_t*>(p.out)[s * p.o_stride_s + h * p.o_stride_h + d] = bits;
 }
 
-template <KvType KV, QType QT, int D, int NT, int KIND>
+template <KvType KV, QType QT, int D, int NT, int KIND, int OCC>
 cudaError_t launch_one(const CUtensorMap& km, const CUtensorMap& vm, const DecodeParams& p, cudaStream_t st) {
-  using C = Cfg<KV, QT, D, NT, KIND>;
-  auto kern = decode_kernel<KV, QT, D, NT, KIND>;
+  using C = Cfg<KV, QT, D, NT, KIND, OCC>;
+  auto kern = decode_kernel<KV, QT, D, NT, KIND, OCC>;
   static int configured_devices = 0;  // bit per device
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (dev < 31 && !(__atomic_load_n(&configured_devices, __ATOMIC_ACQUIRE) & (1 << dev))) {
+  if (dev >= 31 || !(__atomic_load_n(&configured_devices, __ATOMIC_ACQUIRE) & (1 << dev))) {
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return e;
-    __atomic_fetch_or(&configured_devices, 1 << dev, __ATOMIC_ACQ_REL);
-  } else if (dev >= 31) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
-    if (e != cudaSuccess) return e;
+    if (dev < 31) __atomic_fetch_or(&configured_devices, 1 << dev, __ATOMIC_ACQ_REL);
   }
   dim3 grid(p.num_partitions, p.num_kv_heads, p.num_seqs);
   kern<<<grid, C::kThreads, C::kSmemBytes, st>>>(km, vm, p);
   return cudaGetLastError();
 }
 
+// Occupancy per variant (see Cfg): tensor-core e4m3 with one n-tile 4 CTAs/SM, tensor-core 16-bit
+// grouped queries 3, everything else 2.
 template <KvType KV, QType QT, int D, int KIND>
-cudaError_t launch_nt(int nt, const CUtensorMap& km, const CUtensorMap& vm, const DecodeParams& p, cudaStream_t st) {
-  if (nt == 1) return launch_one<KV, QT, D, 1, KIND>(km, vm, p, st);
+cudaError_t launch_nt(int nt, int group, const CUtensorMap& km, const CUtensorMap& vm, const DecodeParams& p,
+                      cudaStream_t st) {
   if constexpr (KIND == 1) {
-    if (nt == 2) return launch_one<KV, QT, D, 2, KIND>(km, vm, p, st);
+    if (nt == 1) {
+      if constexpr (KV == KvType::E4M3) return launch_one<KV, QT, D, 1, 1, 4>(km, vm, p, st);
+      if (group > 1) return launch_one<KV, QT, D, 1, 1, 3>(km, vm, p, st);
+      return launch_one<KV, QT, D, 1, 1, 2>(km, vm, p, st);
+    }
+    if (nt == 2) return launch_one<KV, QT, D, 2, 1, 2>(km, vm, p, st);
+  } else {
+    if (nt == 1) return launch_one<KV, QT, D, 1, 0, 2>(km, vm, p, st);
   }
   return cudaErrorInvalidValue;
 }
 
 template <KvType KV, QType QT, int D>
-cudaError_t launch_kind(const DecodeConfig& c, const CUtensorMap& km, const CUtensorMap& vm, const DecodeParams& p,
-                        cudaStream_t st) {
-  if (c.kernel == 1) return launch_nt<KV, QT, D, 1>(c.ntiles, km, vm, p, st);
-  return launch_nt<KV, QT, D, 0>(c.ntiles, km, vm, p, st);
+cudaError_t launch_kind(const DecodeConfig& c, int group, const CUtensorMap& km, const CUtensorMap& vm,
+                        const DecodeParams& p, cudaStream_t st) {
+  if (c.kernel == 1) return launch_nt<KV, QT, D, 1>(c.ntiles, group, km, vm, p, st);
+  return launch_nt<KV, QT, D, 0>(c.ntiles, group, km, vm, p, st);
 }
 
 }  // namespace
@@ -729,16 +733,17 @@ bool decode_supported(const DecodeConfig& c) {
 cudaError_t launch_decode(const DecodeConfig& c, const CUtensorMap& km, const CUtensorMap& vm, const DecodeParams& p,
                           cudaStream_t st) {
   if (!decode_supported(c)) return cudaErrorInvalidValue;
+  const int g = p.group;
   if (c.kv == KvType::F16) {
-    return c.head_dim == 128 ? launch_kind<KvType::F16, QType::F16, 128>(c, km, vm, p, st)
-                             : launch_kind<KvType::F16, QType::F16, 64>(c, km, vm, p, st);
+    return c.head_dim == 128 ? launch_kind<KvType::F16, QType::F16, 128>(c, g, km, vm, p, st)
+                             : launch_kind<KvType::F16, QType::F16, 64>(c, g, km, vm, p, st);
   }
   if (c.kv == KvType::BF16) {
-    return c.head_dim == 128 ? launch_kind<KvType::BF16, QType::BF16, 128>(c, km, vm, p, st)
-                             : launch_kind<KvType::BF16, QType::BF16, 64>(c, km, vm, p, st);
+    return c.head_dim == 128 ? launch_kind<KvType::BF16, QType::BF16, 128>(c, g, km, vm, p, st)
+                             : launch_kind<KvType::BF16, QType::BF16, 64>(c, g, km, vm, p, st);
   }
-  return c.q == QType::BF16 ? launch_kind<KvType::E4M3, QType::BF16, 128>(c, km, vm, p, st)
-                            : launch_kind<KvType::E4M3, QType::F16, 128>(c, km, vm, p, st);
+  return c.q == QType::BF16 ? launch_kind<KvType::E4M3, QType::BF16, 128>(c, g, km, vm, p, st)
+                            : launch_kind<KvType::E4M3, QType::F16, 128>(c, g, km, vm, p, st);
 }
 
 cudaError_t launch_reduce(const DecodeConfig& c, const DecodeParams& p, cudaStream_t st) {

@@ -70,6 +70,7 @@ struct CacheParams {
 cudaError_t launch_reshape_and_cache(int src_bf16, KvType cache, const CacheParams& p, cudaStream_t stream);
 
 uint32_t* decode_error_word();  // device address of the library's own error word
+
 cudaError_t read_and_clear_error_word(uint32_t* bits, int clear);
 
 }  // namespace pa

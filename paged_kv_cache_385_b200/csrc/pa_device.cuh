@@ -148,10 +148,14 @@ __device__ __forceinline__ float2 unpack2(uint32_t x) {
   }
 }
 
-// Two e4m3 codes (low byte -> low half) to an f16x2 holding their exact values.
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes) {
-  __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two_codes & 0xffffu), __NV_E4M3);
-  return static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
+// Four e4m3 codes (bytes 0..3 of x) to two f16x2 of their exact values: lo = (b0, b1), hi = (b2, b3).
+__device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t x, uint32_t& lo, uint32_t& hi) {
+  asm("{\n\t.reg .b16 a, b;\n\t"
+      "mov.b32 {a, b}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, a;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %1, b;\n\t}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(x));
 }
 
 // Round-to-nearest-even, saturating to +-448, of two floats into two e4m3 codes (lo -> low byte).
