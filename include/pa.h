@@ -150,6 +150,33 @@ int32_t pa_decode_partition_tokens(int32_t num_seqs, int32_t num_kv_heads, int32
 size_t pa_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
                                  int32_t max_context_len, int32_t partition_tokens);
 
+/*
+ * pa_decode_no_alloc -- pa_decode for callers that cannot allocate device memory.
+ * (The vLLM pages have no counterpart to this call; it is a property of this library's interface.)
+ * pa_decode needs a caller-provided workspace whenever it splits contexts into partitions. Some
+ * callers cannot get one: a plugin whose host framework owns all device memory and passes it only
+ * inputs and outputs, a process whose device-memory budget is fixed at start-up, or a serving loop
+ * that cannot afford a cudaMalloc (which may synchronise the whole device) inside a step. This call
+ * is pa_decode with the scratch taken from a static array of PA_NO_ALLOC_SCRATCH_BYTES that the
+ * library keeps in device memory; it allocates nothing and takes no workspace (opts->workspace must
+ * be NULL and workspace_bytes 0, else PA_ERR_INVALID_ARG). All other arguments, results and errors
+ * are those of pa_decode.
+ *   - A batch whose split needs more than PA_NO_ALLOC_SCRATCH_BYTES (see pa_decode_workspace_bytes)
+ *     is rejected with PA_ERR_WORKSPACE before any device work; larger partition_tokens needs less.
+ *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress, with
+ *     that device current) and caches it; make that first call before any stream capture.
+ *   - The array takes PA_NO_ALLOC_SCRATCH_BYTES (32 MiB) on every device where the library's device
+ *     code is loaded (depending on CUDA's module-loading mode, at start-up or at the latest on the
+ *     first call), until the process exits.
+ *   - All calls on a device share the array and it keeps the last call's contents (nothing in it
+ *     needs to start at zero). Calls whose kernels overlap on the GPU, e.g. on two unordered
+ *     streams, race on it: order them on one stream.
+ */
+#define PA_NO_ALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+int pa_decode_no_alloc(pa_tensor* out, const pa_tensor* q, const pa_tensor* k_cache, const pa_tensor* v_cache,
+                       const pa_tensor* block_tables, const pa_tensor* context_lens, float scale,
+                       int32_t num_kv_heads, const pa_decode_opts* opts, void* stream);
+
 /* Static string for a pa_status value. */
 const char* pa_status_string(int status);
 

@@ -76,6 +76,7 @@ def _load() -> ctypes.CDLL:
         "pa_decode_opts_init": (None, [ctypes.POINTER(PaDecodeOpts)]),
         "pa_reshape_and_cache": (ctypes.c_int, [P, P, P, P, P, F32, F32, VP]),
         "pa_decode": (ctypes.c_int, [P, P, P, P, P, P, F32, I32, ctypes.POINTER(PaDecodeOpts), VP]),
+        "pa_decode_no_alloc": (ctypes.c_int, [P, P, P, P, P, P, F32, I32, ctypes.POINTER(PaDecodeOpts), VP]),
         "pa_decode_partition_tokens": (I32, [I32, I32, I32]),
         "pa_decode_workspace_bytes": (SZ, [I32, I32, I32, I32, I32, I32]),
         "pa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -192,6 +193,30 @@ def pa_decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache
             as_pa_tensor(context_lens, "context_lens")]
     _check(_lib.pa_decode(*[ctypes.byref(a) for a in args], float(scale), int(num_kv_heads), ctypes.byref(opts),
                           ctypes.c_void_p(_stream_handle(stream))), "pa_decode")
+
+
+# Size of the library's built-in scratch array used by pa_decode_no_alloc (PA_NO_ALLOC_SCRATCH_BYTES).
+NO_ALLOC_SCRATCH_BYTES = 32 << 20
+
+
+def pa_decode_no_alloc(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                       block_tables: torch.Tensor, context_lens: torch.Tensor, scale: float, num_kv_heads: int,
+                       opts: Optional[PaDecodeOpts] = None, stream=None, **kw) -> None:
+    """pa_decode for callers that cannot allocate device memory (see ``pa_decode_no_alloc`` in include/pa.h).
+
+    The split-partition scratch comes from a fixed array inside the library, so no ``workspace``
+    may be passed. Batches needing more than ``NO_ALLOC_SCRATCH_BYTES`` of scratch are rejected.
+    """
+    if opts is None:
+        opts = decode_opts(**kw)
+    elif kw:
+        raise TypeError("pass either opts or keyword options, not both")
+    args = [as_pa_tensor(out, "out"), as_pa_tensor(q, "q"), as_pa_tensor(k_cache, "k_cache"),
+            as_pa_tensor(v_cache, "v_cache"), as_pa_tensor(block_tables, "block_tables"),
+            as_pa_tensor(context_lens, "context_lens")]
+    _check(_lib.pa_decode_no_alloc(*[ctypes.byref(a) for a in args], float(scale), int(num_kv_heads),
+                                   ctypes.byref(opts), ctypes.c_void_p(_stream_handle(stream))),
+           "pa_decode_no_alloc")
 
 
 def pa_decode_partition_tokens(num_seqs: int, num_kv_heads: int, max_context_len: int) -> int:

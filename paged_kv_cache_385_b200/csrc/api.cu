@@ -150,6 +150,18 @@ size_t workspace_layout(int64_t B, int64_t Hq, int64_t D, int64_t P, size_t* ml_
 
 }  // namespace
 
+namespace pa {
+int set_last_error(int status, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return status;
+}
+}  // namespace pa
+
 extern "C" {
 
 const char* pa_version(void) { return "0.1.0"; }

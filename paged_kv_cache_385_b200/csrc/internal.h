@@ -71,6 +71,8 @@ cudaError_t launch_reshape_and_cache(int src_bf16, KvType cache, const CachePara
 
 uint32_t* decode_error_word();  // device address of the library's own error word
 
+// Record the reason pa_last_error() reports for this thread; returns status.
+int set_last_error(int status, const char* fmt, ...);
 cudaError_t read_and_clear_error_word(uint32_t* bits, int clear);
 
 }  // namespace pa
