@@ -41,12 +41,15 @@ FALLBACK_HBM_GBS = 6650.0
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--steps", type=int, default=3000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="llama7b_mha", choices=sorted(W.FULL))
     ap.add_argument("--kernel", type=int, default=-1, help="-1 library choice, 0 CUDA-core, 1 tensor-core")
     ap.add_argument("--partition-tokens", type=int, default=None)
+    ap.add_argument("--step", choices=["fused", "separate"], default="fused",
+                    help="fused: pa_decode_step (new-token write inside the decode launch); "
+                         "separate: pa_reshape_and_cache then pa_decode")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args()
@@ -177,6 +180,7 @@ class Setup:
             eff_pt = 0
         self.split = eff_pt > 0 and -(-self.max_ctx // eff_pt) > 1
         self.partition_tokens_used = eff_pt if self.split else 0
+        self.fused_step = True
         self.launches_per_step = 2 + (1 if self.split else 0)
         torch.cuda.synchronize(device)
 
@@ -189,9 +193,17 @@ class Setup:
         self.pa.pa_decode(self.out, self.q, self.k_cache, self.v_cache, self.bt, self.lens, w.scale, w.num_kv_heads,
                           opts=self.opts, stream=stream)
 
+    def fused(self, stream=None):
+        w = self.w
+        self.pa.pa_decode_step(self.out, self.q, self.new_k, self.new_v, self.new_slots, self.k_cache, self.v_cache,
+                               self.bt, self.lens, w.scale, w.num_kv_heads, opts=self.opts, stream=stream)
+
     def step(self):
-        self.k1()
-        self.decode()
+        if self.fused_step:
+            self.fused()
+        else:
+            self.k1()
+            self.decode()
 
 
 def measured_hbm_peak():
@@ -272,6 +284,8 @@ def run_ours(args, rank, world, local_rank):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
     w = W.FULL[args.workload]
     st = Setup(w, device, args.kernel, args.partition_tokens)
+    st.fused_step = args.step == "fused"
+    st.launches_per_step = (1 if st.fused_step else 2) + (1 if st.split else 0)
     kv_bytes = W.kv_bytes_read(w, st.lens_host)
     K, Wm = args.steps, max(3, args.warmup)
 
@@ -285,25 +299,37 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize(device)
     pa.pa_read_device_error(clear=True)
 
-    # ---- device-timed steps, with per-launch events for the decode call --------------------------
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    # ---- device-timed steps ------------------------------------------------------------------
+    # Only the region is bracketed by events: an event between two launches serialises them (the
+    # next launch can no longer overlap the previous one's tail) and adds ~9 us per step. A fused
+    # step is one decode launch (plus the partition merge when the context is split), so the
+    # per-launch duration of the decode call is the region's time over K. In "separate" mode a
+    # second pass of K steps brackets each pa_decode with events to isolate it.
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize(device)
     with ClockSampler(local_rank) as clocks:
         start.record()
+        for _ in range(K):
+            st.step()
+        end.record()
+        torch.cuda.synchronize(device)
+    barrier()
+    total_ms = start.elapsed_time(end)
+    k1_ms = []
+    if st.fused_step:
+        dec_ms = [total_ms / K]
+    else:
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
         for k in range(K):
             ev[k][0].record()
             st.k1()
             ev[k][1].record()
             st.decode()
             ev[k][2].record()
-        end.record()
         torch.cuda.synchronize(device)
-    barrier()
-    total_ms = start.elapsed_time(end)
-    dec_ms = [ev[k][1].elapsed_time(ev[k][2]) for k in range(K)]
-    k1_ms = [ev[k][0].elapsed_time(ev[k][1]) for k in range(K)]
+        dec_ms = [ev[k][1].elapsed_time(ev[k][2]) for k in range(K)]
+        k1_ms = [ev[k][0].elapsed_time(ev[k][1]) for k in range(K)]
     dev_err = pa.pa_read_device_error(clear=True)
     if world > 1:
         import torch.distributed as dist
@@ -379,7 +405,9 @@ def run_ours(args, rank, world, local_rank):
         "ms_per_step": round(ms_per_step, 5),
         "us_per_step": round(ms_per_step * 1e3, 2),
         "us_decode": round(dec_avg_s * 1e6, 2),
-        "us_reshape_and_cache": round(statistics.mean(k1_ms) * 1e3, 2),
+        "us_reshape_and_cache": round(statistics.mean(k1_ms) * 1e3, 2) if k1_ms else None,
+        "step": "pa_decode_step (new-token write fused into the decode launch)" if st.fused_step
+                else "pa_reshape_and_cache + pa_decode",
         "pct_of_8TBps": round(100.0 * value / world / 8000.0, 1),
         "higher_is_better": True,
         "scaling": "weak",
@@ -393,9 +421,13 @@ def run_ours(args, rank, world, local_rank):
                    "partition_tokens": st.partition_tokens_used, "kernel": "tensor-core" if args.kernel != 0 else "cuda-core",
                    "l2": f"inputs larger than L2: {kv_bytes / 1e9:.2f} GB of KV per step vs 126 MB L2, no flush",
                    "parallelism": f"replicas x{world}"},
-        "roofline": {"bound": "hbm", "kernel": "pa_decode (decode kernel" + (" + partition merge)" if st.split else ")"),
+        "roofline": {"bound": "hbm", "kernel": ("pa_decode_step" if st.fused_step else "pa_decode")
+                     + (" (decode kernel + partition merge)" if st.split else " (decode kernel)"),
                      "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic, "peak_source": peak_src,
+                     "launch_us": round(dec_avg_s * 1e6, 2),
+                     "launch_timing": ("CUDA events around the K-step timed region / K (one decode call per step)"
+                                       if st.fused_step else "CUDA events around each pa_decode, second pass of K steps"),
                      "algorithmic_bytes_per_launch": kv_bytes},
         "cpu_baseline": cpu,
         "e2e": e2e,

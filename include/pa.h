@@ -139,6 +139,23 @@ int pa_decode(pa_tensor* out, const pa_tensor* q, const pa_tensor* k_cache, cons
               const pa_tensor* block_tables, const pa_tensor* context_lens, float scale, int32_t num_kv_heads,
               const pa_decode_opts* opts, void* stream);
 
+/*
+ * pa_decode_step -- pa_reshape_and_cache of one new token per sequence followed by pa_decode, in one
+ * launch: the CTA that reads a sequence's last page writes the new token's K/V row (for its KV head)
+ * into the slot first, then decodes. Same results, pool bytes and errors as the two calls in order.
+ *   key, value    [B, Hkv, D] device F16/BF16 (last stride 1, 16-B aligned rows): the token at position
+ *                 context_lens[s] - 1 of sequence s.
+ *   slot_mapping  [B] device I64: its slot, which must lie in the page that block_tables[s] maps
+ *                 position context_lens[s] - 1 to (the normal decode step), or -1 to skip.
+ *   Other arguments as pa_decode; opts->k_scale/v_scale also quantise the e4m3 write.
+ * Source: vLLM notes page, "PagedAttention / Cache Engine" (write a position's page) and "内核优化";
+ * fusing the two calls is this library's choice.
+ */
+int pa_decode_step(pa_tensor* out, const pa_tensor* q, const pa_tensor* key, const pa_tensor* value,
+                   const pa_tensor* slot_mapping, pa_tensor* k_cache, pa_tensor* v_cache,
+                   const pa_tensor* block_tables, const pa_tensor* context_lens, float scale, int32_t num_kv_heads,
+                   const pa_decode_opts* opts, void* stream);
+
 /* Partition size pa_decode uses when opts->partition_tokens == 0 and a workspace is given
  * (0 = no split: the batch's B * Hkv (sequence, KV head) units already fill the GPU and every
  * context fits one CTA, <= 2048 tokens). Otherwise the largest of 2048, 1024, 512 that still gives

@@ -76,6 +76,7 @@ def _load() -> ctypes.CDLL:
         "pa_decode_opts_init": (None, [ctypes.POINTER(PaDecodeOpts)]),
         "pa_reshape_and_cache": (ctypes.c_int, [P, P, P, P, P, F32, F32, VP]),
         "pa_decode": (ctypes.c_int, [P, P, P, P, P, P, F32, I32, ctypes.POINTER(PaDecodeOpts), VP]),
+        "pa_decode_step": (ctypes.c_int, [P, P, P, P, P, P, P, P, P, F32, I32, ctypes.POINTER(PaDecodeOpts), VP]),
         "pa_decode_no_alloc": (ctypes.c_int, [P, P, P, P, P, P, F32, I32, ctypes.POINTER(PaDecodeOpts), VP]),
         "pa_decode_partition_tokens": (I32, [I32, I32, I32]),
         "pa_decode_workspace_bytes": (SZ, [I32, I32, I32, I32, I32, I32]),
@@ -193,6 +194,23 @@ def pa_decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache
             as_pa_tensor(context_lens, "context_lens")]
     _check(_lib.pa_decode(*[ctypes.byref(a) for a in args], float(scale), int(num_kv_heads), ctypes.byref(opts),
                           ctypes.c_void_p(_stream_handle(stream))), "pa_decode")
+
+
+def pa_decode_step(out: torch.Tensor, q: torch.Tensor, key: torch.Tensor, value: torch.Tensor,
+                   slot_mapping: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                   block_tables: torch.Tensor, context_lens: torch.Tensor, scale: float, num_kv_heads: int,
+                   opts: Optional[PaDecodeOpts] = None, stream=None, **kw) -> None:
+    """pa_reshape_and_cache of one new token per sequence + pa_decode in one launch (include/pa.h)."""
+    if opts is None:
+        opts = decode_opts(**kw)
+    elif kw:
+        raise TypeError("pass either opts or keyword options, not both")
+    args = [as_pa_tensor(out, "out"), as_pa_tensor(q, "q"), as_pa_tensor(key, "key"), as_pa_tensor(value, "value"),
+            as_pa_tensor(slot_mapping, "slot_mapping"), as_pa_tensor(k_cache, "k_cache"),
+            as_pa_tensor(v_cache, "v_cache"), as_pa_tensor(block_tables, "block_tables"),
+            as_pa_tensor(context_lens, "context_lens")]
+    _check(_lib.pa_decode_step(*[ctypes.byref(a) for a in args], float(scale), int(num_kv_heads), ctypes.byref(opts),
+                               ctypes.c_void_p(_stream_handle(stream))), "pa_decode_step")
 
 
 # Size of the library's built-in scratch array used by pa_decode_no_alloc (PA_NO_ALLOC_SCRATCH_BYTES).

@@ -282,9 +282,12 @@ int pa_reshape_and_cache(const pa_tensor* key, const pa_tensor* value, const pa_
   return ok();
 }
 
-int pa_decode(pa_tensor* out, const pa_tensor* q, const pa_tensor* k_cache, const pa_tensor* v_cache,
-              const pa_tensor* block_tables, const pa_tensor* context_lens, float scale, int32_t num_kv_heads,
-              const pa_decode_opts* opts_in, void* stream) {
+// pa_decode, and pa_decode_step when new_key/new_value/new_slots are given (the decode kernel then
+// writes each sequence's new token into the cache before reading its pages).
+static int decode_impl(pa_tensor* out, const pa_tensor* q, const pa_tensor* k_cache, const pa_tensor* v_cache,
+                       const pa_tensor* block_tables, const pa_tensor* context_lens, float scale, int32_t num_kv_heads,
+                       const pa_decode_opts* opts_in, void* stream, const pa_tensor* new_key,
+                       const pa_tensor* new_value, const pa_tensor* new_slots) {
   pa_decode_opts opts;
   pa_decode_opts_init(&opts);
   if (opts_in) opts = *opts_in;
@@ -407,6 +410,43 @@ int pa_decode(pa_tensor* out, const pa_tensor* q, const pa_tensor* k_cache, cons
     p.ws_ml = reinterpret_cast<float*>(static_cast<char*>(opts.workspace) + ml_off);
   }
 
+  if (new_key) {
+    if ((st = check_tensor(new_key, "key", 3)) || (st = check_tensor(new_value, "value", 3)) ||
+        (st = check_tensor(new_slots, "slot_mapping", 1)))
+      return st;
+    if (new_key->dtype != PA_F16 && new_key->dtype != PA_BF16)
+      return fail(PA_ERR_INVALID_ARG, "key dtype %s; expected F16 or BF16", dtype_name(new_key->dtype));
+    if (new_value->dtype != new_key->dtype) return fail(PA_ERR_INVALID_ARG, "value dtype differs from key dtype");
+    if (cd != PA_E4M3 && cd != new_key->dtype)
+      return fail(PA_ERR_INVALID_ARG, "cache dtype %s does not match key dtype %s", dtype_name(cd),
+                  dtype_name(new_key->dtype));
+    for (int i = 0; i < 3; ++i) {
+      const int64_t want = i == 0 ? B : (i == 1 ? num_kv_heads : D);
+      if (new_key->shape[i] != want || new_value->shape[i] != want)
+        return fail(PA_ERR_INVALID_ARG, "key/value must be [num_seqs, num_kv_heads, head_dim] (one new token each)");
+    }
+    if (new_slots->dtype != PA_I64 || new_slots->shape[0] != B || (new_slots->stride[0] != 1 && B > 1))
+      return fail(PA_ERR_INVALID_ARG, "slot_mapping must be contiguous I64 [num_seqs]");
+    if (new_key->stride[2] != 1 || new_value->stride[2] != 1 || !aligned(new_key->data, 16) ||
+        !aligned(new_value->data, 16) || new_key->stride[0] % 8 || new_key->stride[1] % 8 ||
+        new_value->stride[0] % 8 || new_value->stride[1] % 8)
+      return fail(PA_ERR_INVALID_ARG, "key/value rows must be contiguous and 16-byte aligned");
+    if (!new_key->data || !new_value->data || !new_slots->data) return fail(PA_ERR_INVALID_ARG, "NULL data pointer");
+    p.new_k = new_key->data;
+    p.new_v = new_value->data;
+    p.nk_stride_s = new_key->stride[0];
+    p.nk_stride_h = new_key->stride[1];
+    p.nv_stride_s = new_value->stride[0];
+    p.nv_stride_h = new_value->stride[1];
+    p.new_slots = static_cast<const int64_t*>(new_slots->data);
+    p.k_cache = k_cache->data;
+    p.v_cache = v_cache->data;
+    p.new_src_bf16 = new_key->dtype == PA_BF16;
+    volatile float one = 1.0f;  // IEEE float32 reciprocals, as pa_reshape_and_cache forms them
+    p.k_inv_scale = cd == PA_E4M3 ? one / k_scale : 1.0f;
+    p.v_inv_scale = cd == PA_E4M3 ? one / v_scale : 1.0f;
+  }
+
   CUtensorMap km, vm;
   const int esz = elem_bytes(cd);
   if ((st = encode_pool_map(&km, k_cache, esz)) || (st = encode_pool_map(&vm, v_cache, esz))) return st;
@@ -418,6 +458,22 @@ int pa_decode(pa_tensor* out, const pa_tensor* q, const pa_tensor* k_cache, cons
     if (e != cudaSuccess) return fail(PA_ERR_CUDA, "reduce launch: %s", cudaGetErrorString(e));
   }
   return ok();
+}
+
+int pa_decode(pa_tensor* out, const pa_tensor* q, const pa_tensor* k_cache, const pa_tensor* v_cache,
+              const pa_tensor* block_tables, const pa_tensor* context_lens, float scale, int32_t num_kv_heads,
+              const pa_decode_opts* opts, void* stream) {
+  return decode_impl(out, q, k_cache, v_cache, block_tables, context_lens, scale, num_kv_heads, opts, stream, nullptr,
+                     nullptr, nullptr);
+}
+
+int pa_decode_step(pa_tensor* out, const pa_tensor* q, const pa_tensor* key, const pa_tensor* value,
+                   const pa_tensor* slot_mapping, pa_tensor* k_cache, pa_tensor* v_cache,
+                   const pa_tensor* block_tables, const pa_tensor* context_lens, float scale, int32_t num_kv_heads,
+                   const pa_decode_opts* opts, void* stream) {
+  if (!key || !value || !slot_mapping) return fail(PA_ERR_INVALID_ARG, "key, value and slot_mapping are required");
+  return decode_impl(out, q, k_cache, v_cache, block_tables, context_lens, scale, num_kv_heads, opts, stream, key,
+                     value, slot_mapping);
 }
 
 }  // extern "C"

@@ -24,6 +24,7 @@
 //    ldmatrix.trans); e4m3 pages are widened to f16 in registers (exact).
 //  * CUDA-core (kernel 0): float32 FMA dot products and axpys, for comparison and for G = 1.
 #include <cfloat>
+#include <utility>
 
 #include "internal.h"
 #include "pa_device.cuh"
@@ -226,10 +227,12 @@ struct TcMath {
           uint32_t a[4];
           e4m3x4_to_f16x2x2(t0, a[0], a[1]);
           e4m3x4_to_f16x2x2(t1, a[2], a[3]);
-          a[0] &= mlo;
-          a[1] &= mlo;
-          a[2] &= mhi;
-          a[3] &= mhi;
+          if (nv < 16) {
+            a[0] &= mlo;
+            a[1] &= mlo;
+            a[2] &= mhi;
+            a[3] &= mhi;
+          }
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt) mma_16816<false>(acc[nt][2 * mp + half], a, pf[nt][0], pf[nt][1]);
         }
@@ -239,10 +242,12 @@ struct TcMath {
       for (int mt = 0; mt < KS; ++mt) {
         uint32_t a[4];
         ldmatrix_x4_trans(a, vb + (mt >> 2) * 2048 + swz(t_tok, ((mt & 3) << 1) + t_co));
-        a[0] &= mlo;
-        a[1] &= mlo;
-        a[2] &= mhi;
-        a[3] &= mhi;
+        if (nv < 16) {
+          a[0] &= mlo;
+          a[1] &= mlo;
+          a[2] &= mhi;
+          a[3] &= mhi;
+        }
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) mma_16816<C::kMmaBf16>(acc[nt][mt], a, pf[nt][0], pf[nt][1]);
       }
@@ -463,6 +468,10 @@ __global__ void __launch_bounds__(Cfg<KV, QT, D, NT, KIND, OCC>::kThreads, Cfg<K
 
   const int part = blockIdx.x, hk = blockIdx.y, s = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // Launched as a programmatic dependent: everything this grid reads may come from the previous
+  // kernel on the stream, so wait for it first. The next kernel (partition merge, next step) is let
+  // in once every CTA has finished its page loop (below), when SM slots start to free up.
+  pdl_wait();
   const int G = p.group;
   const int Hq = p.num_kv_heads * G;
   const int PT = p.partition_tokens;
@@ -476,6 +485,43 @@ __global__ void __launch_bounds__(Cfg<KV, QT, D, NT, KIND, OCC>::kThreads, Cfg<K
   }
   const int nparts = (ctx_eff + PT - 1) / PT;
   if (part >= max(nparts, 1)) return;
+
+  // pa_decode_step: the CTA holding the sequence's last partition writes head hk's new K/V row
+  // (position ctx - 1) into its slot before any of its page copies start. No other CTA reads that
+  // page, and the proxy fence + barrier order the writes before this CTA's TMA loads.
+  if (p.new_k != nullptr && part == max(nparts, 1) - 1) {
+    const int64_t slot = p.new_slots[s];
+    if (slot >= 0 && slot < static_cast<int64_t>(p.num_blocks) * 16) {
+      constexpr int kChunks = D / 8;  // 16-byte input chunks per row
+      for (int c = threadIdx.x; c < 2 * kChunks; c += C::kThreads) {
+        const bool is_v = c >= kChunks;
+        const int d0 = (is_v ? c - kChunks : c) * 8;
+        const uint16_t* src = static_cast<const uint16_t*>(is_v ? p.new_v : p.new_k) +
+                              s * (is_v ? p.nv_stride_s : p.nk_stride_s) + hk * (is_v ? p.nv_stride_h : p.nk_stride_h) +
+                              d0;
+        const uint4 raw = *reinterpret_cast<const uint4*>(src);
+        const int64_t dst = (((slot >> 4) * p.num_kv_heads + hk) * 16 + (slot & 15)) * D + d0;
+        if constexpr (C::kFp8) {
+          const float inv = is_v ? p.v_inv_scale : p.k_inv_scale;
+          const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+          uint32_t codes[2] = {0u, 0u};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float2 f = p.new_src_bf16 ? unpack2<true>(w[i]) : unpack2<false>(w[i]);
+            codes[i >> 1] |= f32x2_to_e4m3x2(__fmul_rn(f.x, inv), __fmul_rn(f.y, inv)) << (16 * (i & 1));
+          }
+          *reinterpret_cast<uint2*>(static_cast<uint8_t*>(is_v ? p.v_cache : p.k_cache) + dst) =
+              make_uint2(codes[0], codes[1]);
+        } else {
+          *reinterpret_cast<uint4*>(static_cast<uint16_t*>(is_v ? p.v_cache : p.k_cache) + dst) = raw;
+        }
+      }
+      fence_proxy_async_global();
+    } else if (slot != -1 && threadIdx.x == 0) {
+      atomicOr(p.err, 2u);
+    }
+    __syncthreads();
+  }
 
   typedef uint16_t out_t;
   if (ctx_eff == 0) {  // empty context: output 0
@@ -594,6 +640,7 @@ __global__ void __launch_bounds__(Cfg<KV, QT, D, NT, KIND, OCC>::kThreads, Cfg<K
     if (lane == 0) atomicOr(p.err, 4u);
   }
   const int any_fail = __syncthreads_or(!ok);
+  pdl_launch_dependents();
 
   // ---- merge the warps in fixed order -----------------------------------------------------
   if constexpr (KIND == 1) {
@@ -649,6 +696,8 @@ __global__ void __launch_bounds__(Cfg<KV, QT, D, NT, KIND, OCC>::kThreads, Cfg<K
 template <int D, bool kBf16>
 __global__ void __launch_bounds__(D) reduce_kernel(const DecodeParams p) {
   const int h = blockIdx.x, s = blockIdx.y, d = threadIdx.x;
+  pdl_wait();  // the partials come from the decode grid just before this one
+  pdl_launch_dependents();
   const int Hq = p.num_kv_heads * p.group;
   const int PT = p.partition_tokens;
   int ctx_eff = min(p.context_lens[s], p.max_blocks * 16);
@@ -675,6 +724,23 @@ __global__ void __launch_bounds__(D) reduce_kernel(const DecodeParams p) {
   static_cast<uint16_t*>(p.out)[s * p.o_stride_s + h * p.o_stride_h + d] = bits;
 }
 
+// Launch with programmatic stream serialisation: the kernel may begin while the previous kernel on
+// the stream finishes; it waits for it in pdl_wait() before reading anything.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 template <KvType KV, QType QT, int D, int NT, int KIND, int OCC>
 cudaError_t launch_one(const CUtensorMap& km, const CUtensorMap& vm, const DecodeParams& p, cudaStream_t st) {
   using C = Cfg<KV, QT, D, NT, KIND, OCC>;
@@ -688,9 +754,8 @@ cudaError_t launch_one(const CUtensorMap& km, const CUtensorMap& vm, const Decod
     if (e != cudaSuccess) return e;
     if (dev < 31) __atomic_fetch_or(&configured_devices, 1 << dev, __ATOMIC_ACQ_REL);
   }
-  dim3 grid(p.num_partitions, p.num_kv_heads, p.num_seqs);
-  kern<<<grid, C::kThreads, C::kSmemBytes, st>>>(km, vm, p);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(p.num_partitions, p.num_kv_heads, p.num_seqs), dim3(C::kThreads), C::kSmemBytes, st,
+                    km, vm, p);
 }
 
 // Occupancy per variant (see Cfg): tensor-core e4m3 with one n-tile 4 CTAs/SM, tensor-core 16-bit
@@ -747,16 +812,13 @@ cudaError_t launch_decode(const DecodeConfig& c, const CUtensorMap& km, const CU
 }
 
 cudaError_t launch_reduce(const DecodeConfig& c, const DecodeParams& p, cudaStream_t st) {
-  dim3 grid(p.num_kv_heads * p.group, p.num_seqs);
+  const dim3 grid(p.num_kv_heads * p.group, p.num_seqs);
   const bool bf = c.q == QType::BF16;
-  if (c.head_dim == 128) {
-    if (bf) reduce_kernel<128, true><<<grid, 128, 0, st>>>(p);
-    else reduce_kernel<128, false><<<grid, 128, 0, st>>>(p);
-  } else {
-    if (bf) reduce_kernel<64, true><<<grid, 64, 0, st>>>(p);
-    else reduce_kernel<64, false><<<grid, 64, 0, st>>>(p);
-  }
-  return cudaGetLastError();
+  if (c.head_dim == 128)
+    return bf ? launch_pdl(reduce_kernel<128, true>, grid, dim3(128), 0, st, p)
+              : launch_pdl(reduce_kernel<128, false>, grid, dim3(128), 0, st, p);
+  return bf ? launch_pdl(reduce_kernel<64, true>, grid, dim3(64), 0, st, p)
+            : launch_pdl(reduce_kernel<64, false>, grid, dim3(64), 0, st, p);
 }
 
 uint32_t* decode_error_word() {

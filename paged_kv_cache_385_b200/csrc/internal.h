@@ -31,6 +31,15 @@ struct DecodeParams {
   float* ws_acc;             // [B, Hq, P, D] un-normalised partial outputs (split only)
   float* ws_ml;              // [B, Hq, P, 2] partial (running max in log2 units, sum) (split only)
   uint32_t* err;             // error word (never null)
+  // Fused new-token write (pa_decode_step); new_k == nullptr for plain pa_decode.
+  const void* new_k;         // [B, Hkv, D] f16/bf16
+  const void* new_v;
+  int64_t nk_stride_s, nk_stride_h, nv_stride_s, nv_stride_h;
+  const int64_t* new_slots;  // [B] slot of position ctx - 1, or -1
+  void* k_cache;
+  void* v_cache;
+  int32_t new_src_bf16;
+  float k_inv_scale, v_inv_scale;  // e4m3 caches
 };
 
 struct DecodeConfig {

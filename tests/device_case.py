@@ -112,6 +112,18 @@ class DeviceCase:
         self.write_new_token()
         return self.decode(**kw)
 
+    def step_fused(self, kernel: int = -1, partition_tokens: Optional[int] = None,
+                   out: Optional[torch.Tensor] = None) -> torch.Tensor:
+        """pa_decode_step: the new-token write and the decode in one launch."""
+        w = self.w
+        pt = w.partition_tokens if partition_tokens is None else partition_tokens
+        out = self.out if out is None else out
+        pa.pa_decode_step(out, self.q, self.new_k, self.new_v, self.new_slots, self.k_cache, self.v_cache, self.bt,
+                          self.lens, w.scale, w.num_kv_heads, k_scale=self.k_scale, v_scale=self.v_scale,
+                          max_context_len=self.max_ctx, partition_tokens=pt, workspace=self.workspace(pt),
+                          kernel=kernel)
+        return out
+
     def pool_bytes(self):
         """(k, v) pools as host uint8 [NB, Hkv, 16, D * elem]."""
         w = self.w

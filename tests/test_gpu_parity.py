@@ -77,6 +77,36 @@ def pa_error():
     return pa.pa_read_device_error(clear=True)
 
 
+@pytest.mark.parametrize("name", SMALL)
+def test_fused_step_equals_separate_calls(name):
+    """pa_decode_step == pa_reshape_and_cache then pa_decode: identical pool bytes and output bits."""
+    case, want = oracle(name)
+    w = W.ALL[name]
+    sep = DeviceCase(w)
+    fus = DeviceCase(w)
+    for kernel in _kernels(w):
+        for pt in sorted({w.partition_tokens, 0, 48, 512}):
+            a = sep.step(kernel=kernel, partition_tokens=pt).clone()
+            b = fus.step_fused(kernel=kernel, partition_tokens=pt).clone()
+            torch.cuda.synchronize()
+            assert torch.equal(a.view(torch.int16), b.view(torch.int16)), (kernel, pt)
+            assert max_err(b, want) <= TOL[w.kv_dtype]
+    ka, va = sep.pool_bytes()
+    kb, vb = fus.pool_bytes()
+    assert np.array_equal(ka, kb) and np.array_equal(va, vb)
+    assert np.array_equal(kb, case.k_pool) and np.array_equal(vb, case.v_pool)
+
+
+def test_fused_step_writes_the_token_it_reads():
+    """Before the step the new token's slot holds sentinel bytes; a fused step must still match the oracle."""
+    w = W.ALL["llama3_8b_gqa_small"]
+    _, want = oracle(w.name)
+    dev = DeviceCase(w)  # history only: the new tokens are not in the pool yet
+    out = dev.step_fused(kernel=1)
+    torch.cuda.synchronize()
+    assert max_err(out, want) <= TOL[w.kv_dtype]
+
+
 @pytest.mark.parametrize("name", ["tiny", "llama3_8b_gqa_small", "long70b_fp8_small", "mqa_small"])
 def test_permuted_physical_blocks_give_bit_identical_output(name):
     w = W.ALL[name]
