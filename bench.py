@@ -50,6 +50,9 @@ def parse():
     ap.add_argument("--step", choices=["fused", "separate"], default="fused",
                     help="fused: pa_decode_step (new-token write inside the decode launch); "
                          "separate: pa_reshape_and_cache then pa_decode")
+    ap.add_argument("--op", choices=["step", "copy_blocks", "kv_utilization"], default="step",
+                    help="step: the decode step (the headline); copy_blocks: copy-on-write block copies; "
+                         "kv_utilization: KV memory utilisation of the block allocator (host only)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args()
@@ -469,9 +472,111 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def run_copy_blocks(args, rank, world, local_rank):
+    """Throughput of pa_copy_blocks on the workload's pool: 1024 distinct (src, dst) block pairs per call."""
+    import paged_kv_cache_385_b200 as pa
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    w = W.FULL[args.workload]
+    shape = (w.num_blocks, w.num_kv_heads, w.block_size, w.head_dim)
+    kc = torch.zeros(shape, dtype=TORCH_KV[w.kv_dtype], device=device)
+    vc = torch.zeros_like(kc)
+    n = min(1024, w.num_blocks // 2)
+    perm = torch.randperm(w.num_blocks, generator=torch.Generator().manual_seed(w.seed))
+    mapping = torch.stack([perm[:n], perm[n:2 * n]], dim=1).to(torch.int64).to(device)
+    block_bytes = w.num_kv_heads * w.block_size * w.head_dim * w.kv_elem_bytes
+    moved = n * block_bytes * 2 * 2  # K and V, read + write
+    K, Wm = args.steps, max(3, args.warmup)
+    for _ in range(Wm):
+        pa.pa_copy_blocks(kc, vc, mapping)
+    torch.cuda.synchronize(device)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clocks:
+        a.record()
+        for _ in range(K):
+            pa.pa_copy_blocks(kc, vc, mapping)
+        b.record()
+        torch.cuda.synchronize(device)
+    ms = a.elapsed_time(b) / K
+    peak, peak_src = measured_hbm_peak()
+    gbs = moved / (ms / 1e3) / 1e9
+    if rank == 0:
+        print(json.dumps({
+            "metric": "pa_copy_blocks (copy-on-write block copies): HBM GB/s read+write", "value": round(gbs, 1),
+            "unit": "GB/s", "n_gpus": 1, "steps": K, "warmup": Wm, "ms_per_step": round(ms, 5),
+            "higher_is_better": True, "dtype": w.kv_dtype, "data": "synthetic",
+            "config": {"workload": w.name, "pairs_per_call": n, "block_bytes_per_cache": block_bytes,
+                       "bytes_moved_per_call": moved},
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
+                         "frac": round(gbs / peak, 4), "traffic": None, "peak_source": peak_src},
+            "gpu_launches": K, "clocks": clocks.summary()}), flush=True)
+
+
+def kv_utilization_sim(num_blocks: int = 65536, slots: int = 256, num_requests: int = 4000, seed: int = 7,
+                       reserve_tokens: int = 2048, sample_every: int = 16):
+    """Continuous batching over a synthetic request stream with the library's allocator.
+
+    Up to `slots` sequences run at once; each step every running sequence appends one token (a new
+    block when it crosses a 16-token boundary); finished sequences free their blocks and the next
+    request takes the slot (its prompt blocks allocated at once). Every `sample_every` steps the
+    live token counts and the allocator's blocks in use are recorded. Returns the samples as
+    (live token counts, blocks in use) pairs.
+    """
+    import paged_kv_cache_385_b200 as pa
+    prompts, outs = W.request_stream(seed, num_requests, reserve_tokens)
+    alloc = pa.BlockAllocator(num_blocks)
+    nxt = 0
+    running = []  # [tokens, remaining, blocks]
+    samples = []
+    step = 0
+    while nxt < num_requests or running:
+        while len(running) < slots and nxt < num_requests:
+            n = prompts[nxt]
+            blocks = alloc.alloc_n(-(-n // 16)).tolist()
+            running.append([n, outs[nxt], blocks])
+            nxt += 1
+        for r in running:
+            if r[0] % 16 == 0:
+                r[2].append(alloc.alloc())
+            r[0] += 1
+            r[1] -= 1
+        done = [r for r in running if r[1] <= 0]
+        for r in done:
+            alloc.free_n(torch.tensor(r[2], dtype=torch.int32))
+        running = [r for r in running if r[1] > 0]
+        if step % sample_every == 0 and running:
+            samples.append(([r[0] for r in running], num_blocks - alloc.num_free))
+        step += 1
+    return samples
+
+
+def run_kv_utilization(args, rank):
+    if rank != 0:
+        return
+    t0 = time.perf_counter()
+    samples = kv_utilization_sim()
+    wall = time.perf_counter() - t0
+    tokens = sum(sum(n) for n, _ in samples)
+    held = sum(b * 16 for _, b in samples)
+    reserved = sum(len(n) * 2048 for n, _ in samples)
+    print(json.dumps({
+        "metric": "KV memory utilisation: tokens stored / KV slots held (paged, blocks of 16 on demand)",
+        "value": round(100.0 * tokens / held, 2), "unit": "%", "higher_is_better": True, "data": "synthetic",
+        "contiguous_reservation_pct": round(100.0 * tokens / reserved, 2),
+        "config": {"requests": 4000, "concurrent_slots": 256, "prompt": "U[16,1024]", "output": "exp(mean 256)",
+                   "reserve_tokens_contiguous": 2048, "samples": len(samples)},
+        "wall_s": round(wall, 2)}), flush=True)
+
+
 def main():
     args = parse()
     rank, world, local_rank = dist_env()
+    if args.op == "kv_utilization":
+        run_kv_utilization(args, rank)
+        return 0
+    if args.op == "copy_blocks":
+        run_copy_blocks(args, rank, world, local_rank)
+        return 0
     if args.impl == "reference":
         run_reference(args, rank, world)
         return 0

@@ -156,6 +156,17 @@ int pa_decode_step(pa_tensor* out, const pa_tensor* q, const pa_tensor* key, con
                    const pa_tensor* block_tables, const pa_tensor* context_lens, float scale, int32_t num_kv_heads,
                    const pa_decode_opts* opts, void* stream);
 
+/*
+ * pa_copy_blocks -- copy whole physical blocks (every KV head, K and V caches) for copy-on-write.
+ *   k_cache, v_cache  [num_blocks, Hkv, 16, D] contiguous, same dtype and shape.
+ *   block_mapping     [N, 2] device I64: (src, dst) block ids. Destinations must be distinct and not
+ *                     also sources in the same call (pairs run concurrently). src == dst is a no-op;
+ *                     an id outside [0, num_blocks) skips the pair and sets PA_DEVERR_BAD_BLOCK.
+ * Source: "vLLM 前世今生" section 3.2 (several sequences point at one physical block; copy-on-write
+ * on write). Use with pa_block_cow. N == 0 is a no-op.
+ */
+int pa_copy_blocks(pa_tensor* k_cache, pa_tensor* v_cache, const pa_tensor* block_mapping, void* stream);
+
 /* Partition size pa_decode uses when opts->partition_tokens == 0 and a workspace is given
  * (0 = no split: the batch's B * Hkv (sequence, KV head) units already fill the GPU and every
  * context fits one CTA, <= 2048 tokens). Otherwise the largest of 2048, 1024, 512 that still gives
@@ -230,6 +241,12 @@ int32_t pa_block_alloc(pa_allocator* a);
 int pa_block_incref(pa_allocator* a, int32_t block);
 /* Drop a reference; at 0 the block returns to the free list. PA_ERR_BAD_BLOCK if not allocated. */
 int pa_block_free(pa_allocator* a, int32_t block);
+/* Copy-on-write before writing into `block`: with one reference, *out_block = block and 0 is
+ * returned (write in place). Shared, a fresh block is allocated, the caller's reference moves to it
+ * (block's count drops by one, the new block's is 1), *out_block = the new id and 1 is returned: copy
+ * the page with pa_copy_blocks before writing. PA_ERR_EXHAUSTED (nothing changed) if no block is
+ * free; PA_ERR_BAD_BLOCK if `block` is not allocated. Source: "vLLM 前世今生" section 3.2. */
+int pa_block_cow(pa_allocator* a, int32_t block, int32_t* out_block);
 /* Reference count of a block (0 = free), or PA_ERR_BAD_BLOCK for an id outside the pool. */
 int32_t pa_block_refcount(const pa_allocator* a, int32_t block);
 int32_t pa_allocator_num_free(const pa_allocator* a);

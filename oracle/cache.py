@@ -61,3 +61,18 @@ def pool_values(pool: np.ndarray, kv_dtype: str, scale: float = 1.0) -> np.ndarr
     if kv_dtype == "e4m3":
         return e4m3.dequantize(pool, scale)
     raise ValueError(kv_dtype)
+
+
+def copy_blocks(k_pool: np.ndarray, v_pool: np.ndarray, mapping):
+    """Return new pools where block dst holds block src's bytes, for each (src, dst) pair.
+
+    The pairs are applied to the pools as they were before the call (all sources read first), the
+    reading the copy kernel implements for mappings whose destinations are distinct and are not
+    also sources.
+    """
+    k_out = k_pool.copy()
+    v_out = v_pool.copy()
+    for src, dst in np.asarray(mapping, dtype=np.int64).reshape(-1, 2).tolist():
+        k_out[dst] = k_pool[src]
+        v_out[dst] = v_pool[src]
+    return k_out, v_out

@@ -18,7 +18,10 @@ Readings taken where the pages are silent:
   a given order;
 * a block shared by several sequences carries a reference count, and returns to
   the free list when the count falls to zero;
-* unused block-table entries hold -1.
+* unused block-table entries hold -1;
+* copy-on-write (前世今生 §3.2 names it for shared blocks): before a sequence writes into a block
+  that other sequences also reference, it takes a fresh block, copies the page into it and moves
+  its reference there.
 """
 from __future__ import annotations
 
@@ -69,6 +72,23 @@ class FreeListModel:
             self._stack.append(b)
         return True
 
+    def cow(self, b: int):
+        """Copy-on-write of block b before a write: (block to write, whether its page must be copied).
+
+        With one reference the block is written in place. Shared, the writer's reference moves to a
+        fresh block (b loses one reference), whose page must first receive a copy of b's. None when
+        b is not allocated or no block is free (nothing changes then).
+        """
+        if not (0 <= b < self.num_blocks) or self._ref[b] == 0:
+            return None
+        if self._ref[b] == 1:
+            return b, False
+        nb = self.alloc()
+        if nb is None:
+            return None
+        self._ref[b] -= 1
+        return nb, True
+
     def refcount(self, b: int) -> int:
         return self._ref[b] if 0 <= b < self.num_blocks else -1
 
@@ -117,3 +137,20 @@ def slots_for_positions(block_tables: np.ndarray, seqs: Sequence[int], positions
                         block_size: int = 16) -> np.ndarray:
     """Slot of each (sequence, position) pair, int64."""
     return np.array([slot_of(block_tables[s], p, block_size) for s, p in zip(seqs, positions)], dtype=np.int64)
+
+
+def utilization(token_counts: Sequence[int], block_size: int = 16, reserve_tokens: int = 0):
+    """KV-memory utilisation of live sequences: tokens stored / token slots held.
+
+    Paged (blocks on demand): sum n / sum block_size * ceil(n / block_size); at most block_size - 1
+    slots per sequence are unused. Contiguous reservation of reserve_tokens per sequence (the
+    pre-allocation the pages describe for earlier systems): sum n / (count * reserve_tokens).
+    Source: "vLLM 前世今生" §3.1-3.2 and the notes page "PagedAttention" (pre-allocation waste and
+    fragmentation vs fixed pages allocated on demand).
+    """
+    n = [int(x) for x in token_counts]
+    total = sum(n)
+    held = sum(block_size * (-(-x // block_size)) for x in n)
+    paged = total / held if held else 1.0
+    contiguous = total / (len(n) * reserve_tokens) if (n and reserve_tokens) else None
+    return paged, contiguous

@@ -90,6 +90,8 @@ def _load() -> ctypes.CDLL:
         "pa_block_incref": (ctypes.c_int, [VP, I32]),
         "pa_block_free": (ctypes.c_int, [VP, I32]),
         "pa_block_refcount": (I32, [VP, I32]),
+        "pa_block_cow": (ctypes.c_int, [VP, I32, i32p]),
+        "pa_copy_blocks": (ctypes.c_int, [P, P, P, VP]),
         "pa_allocator_num_free": (I32, [VP]),
         "pa_allocator_num_blocks": (I32, [VP]),
         "pa_blocks_alloc_n": (ctypes.c_int, [VP, I32, i32p]),
@@ -157,6 +159,14 @@ def pa_reshape_and_cache(key: torch.Tensor, value: torch.Tensor, slot_mapping: t
             as_pa_tensor(k_cache, "k_cache"), as_pa_tensor(v_cache, "v_cache")]
     _check(_lib.pa_reshape_and_cache(*[ctypes.byref(a) for a in args], float(k_scale), float(v_scale),
                                      ctypes.c_void_p(_stream_handle(stream))), "pa_reshape_and_cache")
+
+
+def pa_copy_blocks(k_cache: torch.Tensor, v_cache: torch.Tensor, block_mapping: torch.Tensor, stream=None) -> None:
+    """Copy whole blocks (src, dst) of both caches for copy-on-write (see include/pa.h)."""
+    args = [as_pa_tensor(k_cache, "k_cache"), as_pa_tensor(v_cache, "v_cache"),
+            as_pa_tensor(block_mapping, "block_mapping")]
+    _check(_lib.pa_copy_blocks(*[ctypes.byref(a) for a in args], ctypes.c_void_p(_stream_handle(stream))),
+           "pa_copy_blocks")
 
 
 def decode_opts(k_scale: float = 1.0, v_scale: float = 1.0, max_context_len: int = 0, partition_tokens: int = 0,
@@ -337,6 +347,14 @@ class BlockAllocator:
     def free_n(self, blocks: torch.Tensor) -> None:
         b = blocks.to(torch.int32).contiguous()
         _check(_lib.pa_blocks_free_n(self._h, b.numel(), _i32_ptr(b)), "pa_blocks_free_n")
+
+    def cow(self, block: int):
+        """Copy-on-write before writing into ``block``: returns (block_to_write, needs_copy)."""
+        out = ctypes.c_int32(-1)
+        r = int(_lib.pa_block_cow(self._h, int(block), ctypes.byref(out)))
+        if r < 0:
+            _check(r, "pa_block_cow")
+        return int(out.value), r == 1
 
     def refcount(self, block: int) -> int:
         return int(_lib.pa_block_refcount(self._h, int(block)))

@@ -7,7 +7,9 @@
 // the sequences that reference it and returns to the free list when the last one lets go.
 //
 // alloc pops the top of the stack; freeing the last reference pushes the block back on top, so the
-// block released most recently is reused first (warm in L2). No GPU is involved.
+// block released most recently is reused first (warm in L2). Copy-on-write (前世今生 §3.2): a
+// sequence about to write into a block other sequences share moves its reference to a fresh block,
+// whose page the caller fills with pa_copy_blocks first. No GPU is involved.
 #include <cstdint>
 #include <new>
 #include <vector>
@@ -74,6 +76,20 @@ int pa_block_free(pa_allocator* a, int32_t b) {
   if (b < 0 || b >= static_cast<int32_t>(a->ref.size()) || a->ref[b] == 0) return PA_ERR_BAD_BLOCK;
   if (--a->ref[b] == 0) a->stack.push_back(b);
   return PA_OK;
+}
+
+int pa_block_cow(pa_allocator* a, int32_t b, int32_t* out_block) {
+  if (!a || !out_block) return PA_ERR_INVALID_ARG;
+  if (b < 0 || b >= static_cast<int32_t>(a->ref.size()) || a->ref[b] == 0) return PA_ERR_BAD_BLOCK;
+  if (a->ref[b] == 1) {  // sole owner: write in place
+    *out_block = b;
+    return 0;
+  }
+  if (a->stack.empty()) return PA_ERR_EXHAUSTED;
+  const int32_t nb = pa_block_alloc(a);
+  --a->ref[b];
+  *out_block = nb;
+  return 1;
 }
 
 int32_t pa_block_refcount(const pa_allocator* a, int32_t b) {

@@ -460,6 +460,39 @@ static int decode_impl(pa_tensor* out, const pa_tensor* q, const pa_tensor* k_ca
   return ok();
 }
 
+int pa_copy_blocks(pa_tensor* k_cache, pa_tensor* v_cache, const pa_tensor* block_mapping, void* stream) {
+  int st;
+  if ((st = check_tensor(k_cache, "k_cache", 4)) || (st = check_tensor(v_cache, "v_cache", 4)) ||
+      (st = check_tensor(block_mapping, "block_mapping", 2)))
+    return st;
+  if (k_cache->dtype != v_cache->dtype) return fail(PA_ERR_INVALID_ARG, "k_cache and v_cache dtypes differ");
+  for (int i = 0; i < 4; ++i)
+    if (v_cache->shape[i] != k_cache->shape[i]) return fail(PA_ERR_INVALID_ARG, "v_cache shape differs from k_cache");
+  if (k_cache->shape[2] != PA_BLOCK_SIZE) return fail(PA_ERR_INVALID_ARG, "cache shape must be [num_blocks, Hkv, 16, D]");
+  if (!is_contiguous(k_cache) || !is_contiguous(v_cache)) return fail(PA_ERR_INVALID_ARG, "caches must be contiguous");
+  if (block_mapping->dtype != PA_I64 || block_mapping->shape[1] != 2 || !is_contiguous(block_mapping))
+    return fail(PA_ERR_INVALID_ARG, "block_mapping must be contiguous I64 [num_pairs, 2]");
+  const int64_t N = block_mapping->shape[0];
+  if (N == 0) return ok();
+  if (N > 0x7fffffff) return fail(PA_ERR_INVALID_ARG, "too many pairs");
+  const int64_t block_bytes = k_cache->shape[1] * 16 * k_cache->shape[3] * elem_bytes(k_cache->dtype);
+  if (block_bytes % 16) return fail(PA_ERR_UNSUPPORTED, "block size in bytes must be a multiple of 16");
+  if (!aligned(k_cache->data, 16) || !aligned(v_cache->data, 16)) return fail(PA_ERR_INVALID_ARG, "caches must be 16-byte aligned");
+  if (!block_mapping->data) return fail(PA_ERR_INVALID_ARG, "NULL data pointer");
+  pa::CopyParams p{};
+  p.k_cache = k_cache->data;
+  p.v_cache = v_cache->data;
+  p.mapping = static_cast<const int64_t*>(block_mapping->data);
+  p.num_pairs = N;
+  p.block_bytes = block_bytes;
+  p.num_blocks = k_cache->shape[0];
+  p.err = library_error_word();
+  if (!p.err) return fail(PA_ERR_CUDA, "no device error word (no current CUDA device?)");
+  cudaError_t e = pa::launch_copy_blocks(p, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(PA_ERR_CUDA, "copy_blocks launch: %s", cudaGetErrorString(e));
+  return ok();
+}
+
 int pa_decode(pa_tensor* out, const pa_tensor* q, const pa_tensor* k_cache, const pa_tensor* v_cache,
               const pa_tensor* block_tables, const pa_tensor* context_lens, float scale, int32_t num_kv_heads,
               const pa_decode_opts* opts, void* stream) {

@@ -58,7 +58,36 @@ __global__ void __launch_bounds__(128) reshape_and_cache_kernel(const CacheParam
   }
 }
 
+// Copy whole blocks (every KV head, K and V) for copy-on-write: grid (pairs, chunk groups), one
+// 16-byte chunk per thread per cache. Pairs with an id outside the pool are skipped and reported.
+__global__ void __launch_bounds__(256) copy_blocks_kernel(const CopyParams p) {
+  const int64_t pair = blockIdx.x;
+  const int64_t src = p.mapping[2 * pair], dst = p.mapping[2 * pair + 1];
+  if (src < 0 || src >= p.num_blocks || dst < 0 || dst >= p.num_blocks) {
+    if (threadIdx.x == 0 && blockIdx.y == 0) atomicOr(p.err, 1u);
+    return;
+  }
+  if (src == dst) return;
+  const int64_t chunks = p.block_bytes / 16;
+  for (int64_t c = static_cast<int64_t>(blockIdx.y) * blockDim.x + threadIdx.x; c < chunks;
+       c += static_cast<int64_t>(gridDim.y) * blockDim.x) {
+    const uint4* ks = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(p.k_cache) + src * p.block_bytes) + c;
+    const uint4* vs = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(p.v_cache) + src * p.block_bytes) + c;
+    const uint4 kv = *ks, vv = *vs;
+    *(reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.k_cache) + dst * p.block_bytes) + c) = kv;
+    *(reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.v_cache) + dst * p.block_bytes) + c) = vv;
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_copy_blocks(const CopyParams& p, cudaStream_t st) {
+  if (p.num_pairs == 0) return cudaSuccess;
+  const int64_t chunks = p.block_bytes / 16;
+  const unsigned groups = static_cast<unsigned>(std::min<int64_t>(65535, (chunks + 255) / 256));
+  copy_blocks_kernel<<<dim3(static_cast<unsigned>(p.num_pairs), groups), 256, 0, st>>>(p);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_reshape_and_cache(int src_bf16, KvType cache, const CacheParams& p, cudaStream_t st) {
   if (p.num_tokens == 0) return cudaSuccess;

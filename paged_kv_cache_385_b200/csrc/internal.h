@@ -78,6 +78,17 @@ struct CacheParams {
 // src: 0 = f16, 1 = bf16 source; cache: KvType.
 cudaError_t launch_reshape_and_cache(int src_bf16, KvType cache, const CacheParams& p, cudaStream_t stream);
 
+struct CopyParams {
+  void* k_cache;
+  void* v_cache;
+  const int64_t* mapping;  // [N, 2] (src, dst) block ids
+  int64_t num_pairs;
+  int64_t block_bytes;     // bytes of one block of one cache (Hkv * 16 * D * elem)
+  int64_t num_blocks;
+  uint32_t* err;
+};
+cudaError_t launch_copy_blocks(const CopyParams& p, cudaStream_t stream);
+
 uint32_t* decode_error_word();  // device address of the library's own error word
 
 // Record the reason pa_last_error() reports for this thread; returns status.

@@ -71,7 +71,7 @@ def test_null_tensor_is_rejected_without_a_gpu():
 
 
 @settings(max_examples=150, deadline=None)
-@given(n=st.integers(1, 40), ops=st.lists(st.tuples(st.sampled_from("aif"), st.integers(-2, 42)), max_size=150),
+@given(n=st.integers(1, 40), ops=st.lists(st.tuples(st.sampled_from("aifc"), st.integers(-2, 42)), max_size=150),
        seed=st.integers(0, 2**31 - 1))
 def test_allocator_matches_oracle_model(n, ops, seed):
     order = np.random.default_rng(seed).permutation(n).tolist()
@@ -85,6 +85,14 @@ def test_allocator_matches_oracle_model(n, ops, seed):
             assert got == (pa.PA_ERR_EXHAUSTED if want is None else want)
         elif op == "i":
             assert (lib.pa_block_incref(a._h, b) == pa.PA_OK) == model.incref(b)
+        elif op == "c":
+            want = model.cow(b)
+            out = ctypes.c_int32(-7)
+            r = lib.pa_block_cow(a._h, b, ctypes.byref(out))
+            if want is None:
+                assert r in (pa.PA_ERR_BAD_BLOCK, pa.PA_ERR_EXHAUSTED)
+            else:
+                assert (out.value, r == 1) == want
         else:
             assert (lib.pa_block_free(a._h, b) == pa.PA_OK) == model.free(b)
         assert a.num_free == model.num_free

@@ -55,3 +55,14 @@ def test_e4m3_scatter_and_read_back_through_block_table():
         assert np.array_equal(K, e4m3.dequantize(e4m3.quantize(src_k[:, hk], ks), ks))
         V = attention.gather_context(v1, bt[0], n, hk, "e4m3", vs)
         assert np.array_equal(V, e4m3.dequantize(e4m3.quantize(src_v[:, hk], vs), vs))
+
+
+def test_copy_blocks_copies_whole_blocks_only():
+    rng = np.random.default_rng(9)
+    k0, v0 = _pools(rng, 10, 3, 8, 2)
+    mapping = [(2, 7), (5, 0), (9, 9)]
+    k1, v1 = cache.copy_blocks(k0, v0, mapping)
+    for src, dst in mapping:
+        assert np.array_equal(k1[dst], k0[src]) and np.array_equal(v1[dst], v0[src])
+    untouched = [b for b in range(10) if b not in (7, 0)]
+    assert np.array_equal(k1[untouched], k0[untouched]) and np.array_equal(v1[untouched], v0[untouched])

@@ -60,7 +60,7 @@ class _SetModel:
 
 
 @settings(max_examples=200, deadline=None)
-@given(n=st.integers(1, 24), ops=st.lists(st.tuples(st.sampled_from("aif"), st.integers(-2, 26)), max_size=120),
+@given(n=st.integers(1, 24), ops=st.lists(st.tuples(st.sampled_from("aifc"), st.integers(-2, 26)), max_size=120),
        seed=st.integers(0, 2**31 - 1))
 def test_free_list_model_against_set_model(n, ops, seed):
     order = np.random.default_rng(seed).permutation(n).tolist()
@@ -78,14 +78,29 @@ def test_free_list_model_against_set_model(n, ops, seed):
                 assert got is None
         elif op == "i":
             assert fl.incref(b) == ref.incref(b)
+        elif op == "c":
+            before = ref.ref.get(b, 0)
+            got = fl.cow(b)
+            if before == 0:
+                assert got is None
+            elif before == 1:
+                assert got == (b, False)
+            elif not ref.free:
+                assert got is None
+            else:  # the writer's reference moves to a fresh block that must receive a copy
+                nb, copy = got
+                assert copy and nb != b
+                ref.take(nb)
+                handed.append(nb)
+                assert ref.decref(b)
         else:
             assert fl.free(b) == ref.decref(b)
         assert fl.num_free == len(ref.free)
         assert fl.num_free + len(ref.ref) == n
         for blk in range(n):
             assert fl.refcount(blk) == ref.ref.get(blk, 0) >= 0
-    # Until something is freed, blocks come out in the given order.
-    if all(op != "f" for op, _ in ops):
+    # Until something is freed (a copy-on-write also frees a reference), blocks come out in order.
+    if all(op not in "fc" for op, _ in ops):
         assert handed == order[:len(handed)]
 
 

@@ -204,6 +204,19 @@ SMALL: Dict[str, Workload] = {w.name: w for w in (TINY, LLAMA7B_MHA_SMALL, LLAMA
 ALL: Dict[str, Workload] = {**FULL, **SMALL}
 
 
+def request_stream(seed: int, num_requests: int, max_tokens: int = 2048):
+    """Synthetic request mix for the KV-memory utilisation measurement: (prompt, output) lengths.
+
+    Prompts uniform in [16, 1024]; outputs exponential with mean 256, at least 1; prompt + output
+    capped at max_tokens (the length a contiguous allocator would have to reserve).
+    """
+    g = _gen(seed, "requests")
+    prompt = torch.randint(16, 1025, (num_requests,), generator=g)
+    out = (torch.empty(num_requests).exponential_(1.0 / 256.0, generator=g).ceil().clamp(min=1)).to(torch.int64)
+    out = torch.minimum(out, max_tokens - prompt)
+    return prompt.tolist(), out.tolist()
+
+
 def kv_bytes_read(w: Workload, lens: Optional[torch.Tensor] = None) -> int:
     """Algorithmic K+V bytes one decode step reads: sum_s ctx_s * Hkv * D * elem * 2."""
     if lens is None:
