@@ -47,9 +47,10 @@ def parse():
     ap.add_argument("--workload", default="llama7b_mha", choices=sorted(W.FULL))
     ap.add_argument("--kernel", type=int, default=-1, help="-1 library choice, 0 CUDA-core, 1 tensor-core")
     ap.add_argument("--partition-tokens", type=int, default=None)
-    ap.add_argument("--step", choices=["fused", "separate"], default="fused",
+    ap.add_argument("--step", choices=["fused", "separate", "cascade"], default="fused",
                     help="fused: pa_decode_step (new-token write inside the decode launch); "
-                         "separate: pa_reshape_and_cache then pa_decode")
+                         "separate: pa_reshape_and_cache then pa_decode; "
+                         "cascade: pa_decode_cascade over the workload's shared prefix (prefix_gqa)")
     ap.add_argument("--op", choices=["step", "copy_blocks", "kv_utilization"], default="step",
                     help="step: the decode step (the headline); copy_blocks: copy-on-write block copies; "
                          "kv_utilization: KV memory utilisation of the block allocator (host only)")
@@ -184,6 +185,7 @@ class Setup:
         self.split = eff_pt > 0 and -(-self.max_ctx // eff_pt) > 1
         self.partition_tokens_used = eff_pt if self.split else 0
         self.fused_step = True
+        self.cascade_step = False
         self.launches_per_step = 2 + (1 if self.split else 0)
         torch.cuda.synchronize(device)
 
@@ -196,13 +198,27 @@ class Setup:
         self.pa.pa_decode(self.out, self.q, self.k_cache, self.v_cache, self.bt, self.lens, w.scale, w.num_kv_heads,
                           opts=self.opts, stream=stream)
 
+    def cascade(self, stream=None):
+        w = self.w
+        if not hasattr(self, "_casc_opts"):
+            n = self.pa.pa_decode_cascade_workspace_bytes(w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim,
+                                                          self.max_ctx, w.shared_prefix_tokens, 0)
+            self._casc_ws = torch.empty(n, dtype=torch.uint8, device=self.device)
+            self._casc_opts = self.pa.decode_opts(max_context_len=self.max_ctx, workspace=self._casc_ws,
+                                                  kernel=self.kernel)
+        self.pa.pa_decode_cascade(self.out, self.q, self.new_k, self.new_v, self.new_slots, self.k_cache,
+                                  self.v_cache, self.bt, self.lens, w.shared_prefix_tokens, w.scale, w.num_kv_heads,
+                                  opts=self._casc_opts, stream=stream)
+
     def fused(self, stream=None):
         w = self.w
         self.pa.pa_decode_step(self.out, self.q, self.new_k, self.new_v, self.new_slots, self.k_cache, self.v_cache,
                                self.bt, self.lens, w.scale, w.num_kv_heads, opts=self.opts, stream=stream)
 
     def step(self):
-        if self.fused_step:
+        if self.cascade_step:
+            self.cascade()
+        elif self.fused_step:
             self.fused()
         else:
             self.k1()
@@ -287,8 +303,11 @@ def run_ours(args, rank, world, local_rank):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
     w = W.FULL[args.workload]
     st = Setup(w, device, args.kernel, args.partition_tokens)
-    st.fused_step = args.step == "fused"
-    st.launches_per_step = (1 if st.fused_step else 2) + (1 if st.split else 0)
+    st.fused_step = args.step in ("fused", "cascade")
+    st.cascade_step = args.step == "cascade"
+    if st.cascade_step and not w.shared_prefix_tokens:
+        raise SystemExit("--step cascade needs a workload with a shared prefix (prefix_gqa)")
+    st.launches_per_step = 3 if st.cascade_step else (1 if st.fused_step else 2) + (1 if st.split else 0)
     kv_bytes = W.kv_bytes_read(w, st.lens_host)
     K, Wm = args.steps, max(3, args.warmup)
 
@@ -342,23 +361,31 @@ def run_ours(args, rank, world, local_rank):
     ms_per_step = total_ms / K
 
     # ---- end to end through the C ABI with host buffers --------------------------------------
+    # The step's inputs (q, new K/V, slots, block tables, context lengths) are packed into one pinned
+    # host buffer and copied with one H2D copy into a device buffer the step's tensors view; the
+    # output comes back with one D2H copy. The KV pool is the resident cache and is not copied.
     e2e = None
     if not args.no_e2e:
-        hq = st.q.cpu().pin_memory()
-        hk, hv = st.new_k.cpu().pin_memory(), st.new_v.cpu().pin_memory()
-        hs, hbt, hl = st.new_slots.cpu().pin_memory(), st.bt_host.pin_memory(), st.lens_host.pin_memory()
+        parts = [st.q, st.new_k, st.new_v, st.new_slots, st.bt, st.lens]
+        offs, total = [], 0
+        for t in parts:
+            offs.append(total)
+            total += -(-(t.numel() * t.element_size()) // 256) * 256
+        hbuf = torch.empty(total, dtype=torch.uint8).pin_memory()
+        dbuf = torch.empty(total, dtype=torch.uint8, device=device)
+        views = []
+        for t, o in zip(parts, offs):
+            n = t.numel() * t.element_size()
+            hv = hbuf[o:o + n].view(t.dtype).view(t.shape)
+            hv.copy_(t.cpu())
+            views.append(dbuf[o:o + n].view(t.dtype).view(t.shape))
+        st.q, st.new_k, st.new_v, st.new_slots, st.bt, st.lens = views
         hout = torch.empty(st.out.shape, dtype=st.out.dtype).pin_memory()
-        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hs, hbt, hl))
-        d2h = hout.numel() * hout.element_size()
+        h2d, d2h = total, hout.numel() * hout.element_size()
         Ke = max(10, min(K, 500))
 
         def e2e_step():
-            st.q.copy_(hq, non_blocking=True)
-            st.new_k.copy_(hk, non_blocking=True)
-            st.new_v.copy_(hv, non_blocking=True)
-            st.new_slots.copy_(hs, non_blocking=True)
-            st.bt.copy_(hbt, non_blocking=True)
-            st.lens.copy_(hl, non_blocking=True)
+            dbuf.copy_(hbuf, non_blocking=True)
             st.step()
             hout.copy_(st.out, non_blocking=True)
 
@@ -379,10 +406,12 @@ def run_ours(args, rank, world, local_rank):
             t = torch.tensor([e_ms], device=device)
             dist.all_reduce(t, op=dist.ReduceOp.MAX)
             e_ms = float(t.item())
-        e2e = {"value": kv_bytes * world / (e_ms / Ke / 1e3) / 1e9, "unit": "GB/s", "ms_per_step": e_ms / Ke,
-               "steps": Ke, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "note": "per step: pinned H2D of q, new K/V, slots, block tables, context lens; "
-                       "pa_reshape_and_cache + pa_decode; D2H of out. The KV pool is the resident cache."}
+        e2e = {"value": round(kv_bytes * world / (e_ms / Ke / 1e3) / 1e9, 1), "unit": "GB/s",
+               "ms_per_step": round(e_ms / Ke, 5), "steps": Ke, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h,
+               "note": "per step: one pinned H2D copy of the packed inputs (q, new K/V, slots, block tables, "
+                       "context lens), the decode step through the C ABI, one D2H copy of out; the KV pool "
+                       "is the resident cache"}
 
     if world > 1:
         import torch.distributed as dist
@@ -409,8 +438,9 @@ def run_ours(args, rank, world, local_rank):
         "us_per_step": round(ms_per_step * 1e3, 2),
         "us_decode": round(dec_avg_s * 1e6, 2),
         "us_reshape_and_cache": round(statistics.mean(k1_ms) * 1e3, 2) if k1_ms else None,
-        "step": "pa_decode_step (new-token write fused into the decode launch)" if st.fused_step
-                else "pa_reshape_and_cache + pa_decode",
+        "step": ("pa_decode_cascade (shared prefix once per KV head + suffix decode + merge; new-token write fused)"
+                 if st.cascade_step else "pa_decode_step (new-token write fused into the decode launch)"
+                 if st.fused_step else "pa_reshape_and_cache + pa_decode"),
         "pct_of_8TBps": round(100.0 * value / world / 8000.0, 1),
         "higher_is_better": True,
         "scaling": "weak",
@@ -424,8 +454,10 @@ def run_ours(args, rank, world, local_rank):
                    "partition_tokens": st.partition_tokens_used, "kernel": "tensor-core" if args.kernel != 0 else "cuda-core",
                    "l2": f"inputs larger than L2: {kv_bytes / 1e9:.2f} GB of KV per step vs 126 MB L2, no flush",
                    "parallelism": f"replicas x{world}"},
-        "roofline": {"bound": "hbm", "kernel": ("pa_decode_step" if st.fused_step else "pa_decode")
-                     + (" (decode kernel + partition merge)" if st.split else " (decode kernel)"),
+        "roofline": {"bound": "hbm", "kernel": ("pa_decode_cascade (prefix + suffix decode + merge kernels)"
+                                                if st.cascade_step else
+                                                ("pa_decode_step" if st.fused_step else "pa_decode")
+                                                + (" (decode kernel + partition merge)" if st.split else " (decode kernel)")),
                      "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic, "peak_source": peak_src,
                      "launch_us": round(dec_avg_s * 1e6, 2),

@@ -67,6 +67,7 @@ typedef enum pa_dtype { PA_F16 = 0, PA_BF16 = 1, PA_E4M3 = 2, PA_I32 = 3, PA_I64
 #define PA_DEVERR_BAD_SLOT 2u    /* a slot_mapping entry is < -1 or >= num_blocks * 16                       */
 #define PA_DEVERR_TIMEOUT 4u     /* a wait for an asynchronous page copy exceeded its bound                  */
 #define PA_DEVERR_CTX_RANGE 8u   /* context_lens[s] > max_context_len (or > 16 * block-table width)          */
+#define PA_DEVERR_PREFIX 16u     /* pa_decode_cascade: a block table does not share the prefix blocks        */
 
 /* A strided view of caller-owned memory. Strides are in elements, not bytes.
  * Only the first ndim entries of shape/stride are read. The pointer is a
@@ -166,6 +167,33 @@ int pa_decode_step(pa_tensor* out, const pa_tensor* q, const pa_tensor* key, con
  * on write). Use with pa_block_cow. N == 0 is a no-op.
  */
 int pa_copy_blocks(pa_tensor* k_cache, pa_tensor* v_cache, const pa_tensor* block_mapping, void* stream);
+
+/*
+ * pa_decode_cascade -- pa_decode for a batch whose sequences all share their first
+ * shared_prefix_tokens tokens in the same physical blocks (block_tables[s][j] == block_tables[0][j]
+ * for j < shared_prefix_tokens / 16): the shared pages are read once per KV head for all B * G query
+ * rows (a dense tensor-core contraction), each sequence's remaining tokens by the decode kernel, and
+ * the two softmax partials are merged. Same result as pa_decode up to float32 rounding order.
+ *   shared_prefix_tokens  > 0, multiple of 16, <= 16 * block_tables.shape[1]. Sequences shorter than
+ *                 the prefix are fine (their rows stop at their context).
+ *   key, value, slot_mapping  all NULL, or as in pa_decode_step (the new token is written in the same
+ *                 call); a new token must lie past the shared prefix (the prefix blocks are shared
+ *                 and read-only here: copy-on-write them first), else it is skipped with
+ *                 PA_DEVERR_BAD_SLOT.
+ *   F16/BF16 caches only. A workspace is always needed: pa_decode_cascade_workspace_bytes.
+ *   A block table that does not share the prefix blocks sets PA_DEVERR_PREFIX (results undefined).
+ * Source: "vLLM 前世今生" section 3.2 (sequences pointing at the same physical blocks; prefix
+ * sharing) and the notes page's prefix-caching section (a shared prompt prefix computed once).
+ */
+int pa_decode_cascade(pa_tensor* out, const pa_tensor* q, const pa_tensor* key, const pa_tensor* value,
+                      const pa_tensor* slot_mapping, pa_tensor* k_cache, pa_tensor* v_cache,
+                      const pa_tensor* block_tables, const pa_tensor* context_lens, int32_t shared_prefix_tokens,
+                      float scale, int32_t num_kv_heads, const pa_decode_opts* opts, void* stream);
+
+/* Workspace bytes pa_decode_cascade needs (partition_tokens 0 = the library's choice). Host only. */
+size_t pa_decode_cascade_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
+                                         int32_t head_dim, int32_t max_context_len, int32_t shared_prefix_tokens,
+                                         int32_t partition_tokens);
 
 /* Partition size pa_decode uses when opts->partition_tokens == 0 and a workspace is given
  * (0 = no split: the batch's B * Hkv (sequence, KV head) units already fill the GPU and every

@@ -34,6 +34,7 @@ PA_DEVERR_BAD_BLOCK = 1
 PA_DEVERR_BAD_SLOT = 2
 PA_DEVERR_TIMEOUT = 4
 PA_DEVERR_CTX_RANGE = 8
+PA_DEVERR_PREFIX = 16
 
 BLOCK_SIZE = 16
 
@@ -77,6 +78,9 @@ def _load() -> ctypes.CDLL:
         "pa_reshape_and_cache": (ctypes.c_int, [P, P, P, P, P, F32, F32, VP]),
         "pa_decode": (ctypes.c_int, [P, P, P, P, P, P, F32, I32, ctypes.POINTER(PaDecodeOpts), VP]),
         "pa_decode_step": (ctypes.c_int, [P, P, P, P, P, P, P, P, P, F32, I32, ctypes.POINTER(PaDecodeOpts), VP]),
+        "pa_decode_cascade": (ctypes.c_int, [P, P, P, P, P, P, P, P, P, I32, F32, I32,
+                                             ctypes.POINTER(PaDecodeOpts), VP]),
+        "pa_decode_cascade_workspace_bytes": (SZ, [I32, I32, I32, I32, I32, I32, I32]),
         "pa_decode_no_alloc": (ctypes.c_int, [P, P, P, P, P, P, F32, I32, ctypes.POINTER(PaDecodeOpts), VP]),
         "pa_decode_partition_tokens": (I32, [I32, I32, I32]),
         "pa_decode_workspace_bytes": (SZ, [I32, I32, I32, I32, I32, I32]),
@@ -221,6 +225,31 @@ def pa_decode_step(out: torch.Tensor, q: torch.Tensor, key: torch.Tensor, value:
             as_pa_tensor(context_lens, "context_lens")]
     _check(_lib.pa_decode_step(*[ctypes.byref(a) for a in args], float(scale), int(num_kv_heads), ctypes.byref(opts),
                                ctypes.c_void_p(_stream_handle(stream))), "pa_decode_step")
+
+
+def pa_decode_cascade(out: torch.Tensor, q: torch.Tensor, key: Optional[torch.Tensor], value: Optional[torch.Tensor],
+                      slot_mapping: Optional[torch.Tensor], k_cache: torch.Tensor, v_cache: torch.Tensor,
+                      block_tables: torch.Tensor, context_lens: torch.Tensor, shared_prefix_tokens: int, scale: float,
+                      num_kv_heads: int, opts: Optional[PaDecodeOpts] = None, stream=None, **kw) -> None:
+    """Decode with a prefix shared by every sequence read once per KV head (see include/pa.h)."""
+    if opts is None:
+        opts = decode_opts(**kw)
+    elif kw:
+        raise TypeError("pass either opts or keyword options, not both")
+    nk = [None if t is None else ctypes.byref(as_pa_tensor(t, n)) for t, n in
+          ((key, "key"), (value, "value"), (slot_mapping, "slot_mapping"))]
+    args = [as_pa_tensor(out, "out"), as_pa_tensor(q, "q")]
+    rest = [as_pa_tensor(k_cache, "k_cache"), as_pa_tensor(v_cache, "v_cache"),
+            as_pa_tensor(block_tables, "block_tables"), as_pa_tensor(context_lens, "context_lens")]
+    _check(_lib.pa_decode_cascade(*[ctypes.byref(a) for a in args], *nk, *[ctypes.byref(a) for a in rest],
+                                  int(shared_prefix_tokens), float(scale), int(num_kv_heads), ctypes.byref(opts),
+                                  ctypes.c_void_p(_stream_handle(stream))), "pa_decode_cascade")
+
+
+def pa_decode_cascade_workspace_bytes(num_seqs: int, num_q_heads: int, num_kv_heads: int, head_dim: int,
+                                      max_context_len: int, shared_prefix_tokens: int, partition_tokens: int = 0) -> int:
+    return int(_lib.pa_decode_cascade_workspace_bytes(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len,
+                                                      shared_prefix_tokens, partition_tokens))
 
 
 # Size of the library's built-in scratch array used by pa_decode_no_alloc (PA_NO_ALLOC_SCRATCH_BYTES).

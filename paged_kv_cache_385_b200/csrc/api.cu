@@ -287,7 +287,7 @@ int pa_reshape_and_cache(const pa_tensor* key, const pa_tensor* value, const pa_
 static int decode_impl(pa_tensor* out, const pa_tensor* q, const pa_tensor* k_cache, const pa_tensor* v_cache,
                        const pa_tensor* block_tables, const pa_tensor* context_lens, float scale, int32_t num_kv_heads,
                        const pa_decode_opts* opts_in, void* stream, const pa_tensor* new_key,
-                       const pa_tensor* new_value, const pa_tensor* new_slots) {
+                       const pa_tensor* new_value, const pa_tensor* new_slots, int32_t prefix_tokens = 0) {
   pa_decode_opts opts;
   pa_decode_opts_init(&opts);
   if (opts_in) opts = *opts_in;
@@ -370,13 +370,26 @@ static int decode_impl(pa_tensor* out, const pa_tensor* q, const pa_tensor* k_ca
     return fail(PA_ERR_INVALID_ARG, "partition_tokens %lld must be a multiple of 16 in [0, %d]", (long long)pt,
                 pa::kMaxPartitionTokens);
   const bool have_ws = opts.workspace != nullptr && opts.workspace_bytes > 0;
-  if (pt == 0) {
-    pt = auto_partition_tokens(static_cast<int32_t>(B), num_kv_heads, static_cast<int32_t>(max_ctx));
-    if (pt == 0 || (!have_ws && max_ctx <= pa::kMaxPartitionTokens)) pt = std::max<int64_t>(16, (max_ctx + 15) / 16 * 16);
+  // Cascade: the shared prefix goes to the prefix kernel (n_pre chunks); this grid covers the suffix.
+  const bool cascade = prefix_tokens > 0;
+  int64_t n_pre = 0;
+  if (cascade) {
+    if (cd == PA_E4M3) return fail(PA_ERR_UNSUPPORTED, "shared-prefix decode takes F16 or BF16 caches");
+    if (prefix_tokens % 16) return fail(PA_ERR_INVALID_ARG, "shared_prefix_tokens must be a multiple of 16");
+    if (prefix_tokens > max_blocks * 16)
+      return fail(PA_ERR_INVALID_ARG, "shared_prefix_tokens %d exceeds the block-table width", prefix_tokens);
+    n_pre = (prefix_tokens + pa::kPrefixChunkTokens - 1) / pa::kPrefixChunkTokens;
   }
-  int64_t P = (max_ctx + pt - 1) / pt;
+  const int64_t span_max = std::max<int64_t>(max_ctx - (cascade ? prefix_tokens : 0), 0);
+  if (pt == 0) {
+    pt = auto_partition_tokens(static_cast<int32_t>(B), num_kv_heads, static_cast<int32_t>(std::max<int64_t>(span_max, 1)));
+    if (pt == 0 || (!have_ws && span_max <= pa::kMaxPartitionTokens))
+      pt = std::max<int64_t>(16, (std::min<int64_t>(std::max<int64_t>(span_max, 1), pa::kMaxPartitionTokens) + 15) / 16 * 16);
+  }
+  int64_t P = (span_max + pt - 1) / pt;
   if (P < 1) P = 1;
   if (P > 0x7fffffff) return fail(PA_ERR_UNSUPPORTED, "too many partitions");
+  const int64_t ws_parts = n_pre + P;
 
   pa::DecodeParams p{};
   p.out = out->data;
@@ -397,14 +410,19 @@ static int decode_impl(pa_tensor* out, const pa_tensor* q, const pa_tensor* k_ca
   p.num_partitions = static_cast<int32_t>(P);
   p.score_scale_log2 = scale * 1.4426950408889634f * k_scale;
   p.v_scale = v_scale;
+  p.start_tokens = cascade ? prefix_tokens : 0;
+  p.part_offset = static_cast<int32_t>(n_pre);
+  p.ws_parts = static_cast<int32_t>(ws_parts);
+  p.always_partials = cascade ? 1 : 0;
+  p.merge_prefix_inline = cascade && P == 1 ? 1 : 0;
   p.err = opts.error_word ? reinterpret_cast<uint32_t*>(opts.error_word) : library_error_word();
   if (!p.err) return fail(PA_ERR_CUDA, "no device error word (no current CUDA device?)");
-  if (P > 1) {
+  if (ws_parts > 1) {
     size_t ml_off = 0;
-    const size_t need = workspace_layout(B, Hq, D, P, &ml_off);
+    const size_t need = workspace_layout(B, Hq, D, ws_parts, &ml_off);
     if (!have_ws || opts.workspace_bytes < need)
-      return fail(PA_ERR_WORKSPACE, "split into %lld partitions needs a workspace of %zu bytes (got %zu)", (long long)P,
-                  need, have_ws ? opts.workspace_bytes : size_t(0));
+      return fail(PA_ERR_WORKSPACE, "split into %lld partitions needs a workspace of %zu bytes (got %zu)",
+                  (long long)ws_parts, need, have_ws ? opts.workspace_bytes : size_t(0));
     if (!aligned(opts.workspace, 256)) return fail(PA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
     p.ws_acc = static_cast<float*>(opts.workspace);
     p.ws_ml = reinterpret_cast<float*>(static_cast<char*>(opts.workspace) + ml_off);
@@ -451,9 +469,33 @@ static int decode_impl(pa_tensor* out, const pa_tensor* q, const pa_tensor* k_ca
   const int esz = elem_bytes(cd);
   if ((st = encode_pool_map(&km, k_cache, esz)) || (st = encode_pool_map(&vm, v_cache, esz))) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t e = pa::launch_decode(cfg, km, vm, p, s);
+  cudaError_t e;
+  if (cascade) {
+    pa::PrefixParams pp{};
+    pp.q = q->data;
+    pp.q_stride_s = q->stride[0];
+    pp.q_stride_h = q->stride[1];
+    pp.block_tables = p.block_tables;
+    pp.bt_stride = p.bt_stride;
+    pp.context_lens = p.context_lens;
+    pp.num_seqs = p.num_seqs;
+    pp.num_blocks = p.num_blocks;
+    pp.num_kv_heads = num_kv_heads;
+    pp.group = p.group;
+    pp.prefix_tokens = prefix_tokens;
+    pp.chunk_tokens = pa::kPrefixChunkTokens;
+    pp.num_chunks = static_cast<int32_t>(n_pre);
+    pp.score_scale_log2 = p.score_scale_log2;
+    pp.ws_acc = p.ws_acc;
+    pp.ws_ml = p.ws_ml;
+    pp.ws_parts = p.ws_parts;
+    pp.err = p.err;
+    e = pa::launch_prefix(cfg.kv, cfg.head_dim, km, vm, pp, s);
+    if (e != cudaSuccess) return fail(PA_ERR_CUDA, "prefix launch: %s", cudaGetErrorString(e));
+  }
+  e = pa::launch_decode(cfg, km, vm, p, s);
   if (e != cudaSuccess) return fail(PA_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
-  if (P > 1) {
+  if (ws_parts > 1 && !p.merge_prefix_inline) {
     e = pa::launch_reduce(cfg, p, s);
     if (e != cudaSuccess) return fail(PA_ERR_CUDA, "reduce launch: %s", cudaGetErrorString(e));
   }
@@ -498,6 +540,33 @@ int pa_decode(pa_tensor* out, const pa_tensor* q, const pa_tensor* k_cache, cons
               const pa_decode_opts* opts, void* stream) {
   return decode_impl(out, q, k_cache, v_cache, block_tables, context_lens, scale, num_kv_heads, opts, stream, nullptr,
                      nullptr, nullptr);
+}
+
+int pa_decode_cascade(pa_tensor* out, const pa_tensor* q, const pa_tensor* key, const pa_tensor* value,
+                      const pa_tensor* slot_mapping, pa_tensor* k_cache, pa_tensor* v_cache,
+                      const pa_tensor* block_tables, const pa_tensor* context_lens, int32_t shared_prefix_tokens,
+                      float scale, int32_t num_kv_heads, const pa_decode_opts* opts, void* stream) {
+  if (shared_prefix_tokens <= 0) return fail(PA_ERR_INVALID_ARG, "shared_prefix_tokens must be > 0");
+  if ((key == nullptr) != (value == nullptr) || (key == nullptr) != (slot_mapping == nullptr))
+    return fail(PA_ERR_INVALID_ARG, "key, value and slot_mapping are given together or not at all");
+  return decode_impl(out, q, k_cache, v_cache, block_tables, context_lens, scale, num_kv_heads, opts, stream, key,
+                     value, slot_mapping, shared_prefix_tokens);
+}
+
+size_t pa_decode_cascade_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
+                                         int32_t head_dim, int32_t max_context_len, int32_t shared_prefix_tokens,
+                                         int32_t partition_tokens) {
+  if (num_seqs <= 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || shared_prefix_tokens <= 0)
+    return 0;
+  const int64_t n_pre = (shared_prefix_tokens + pa::kPrefixChunkTokens - 1) / pa::kPrefixChunkTokens;
+  const int64_t span = std::max<int64_t>(static_cast<int64_t>(max_context_len) - shared_prefix_tokens, 0);
+  int64_t pt = partition_tokens;
+  if (pt <= 0) {
+    pt = auto_partition_tokens(num_seqs, num_kv_heads, static_cast<int32_t>(std::max<int64_t>(span, 1)));
+    if (pt == 0) pt = std::max<int64_t>(16, (std::min<int64_t>(std::max<int64_t>(span, 1), pa::kMaxPartitionTokens) + 15) / 16 * 16);
+  }
+  const int64_t P = std::max<int64_t>(1, (span + pt - 1) / pt);
+  return workspace_layout(num_seqs, num_q_heads, head_dim, n_pre + P, nullptr);
 }
 
 int pa_decode_step(pa_tensor* out, const pa_tensor* q, const pa_tensor* key, const pa_tensor* value,

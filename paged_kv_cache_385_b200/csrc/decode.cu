@@ -194,12 +194,14 @@ struct TcMath {
       const float2 f0 = unpack2<C::kMmaBf16>(x0), f1 = unpack2<C::kMmaBf16>(x1);
       l[nt][0] = l[nt][0] * al0 + (f0.x + f1.x);
       l[nt][1] = l[nt][1] * al1 + (f0.y + f1.y);
+      if (__any_sync(kFull, al0 != 1.f || al1 != 1.f)) {  // skipped once the running max settles
 #pragma unroll
-      for (int mt = 0; mt < KS; ++mt) {
-        acc[nt][mt][0] *= al0;
-        acc[nt][mt][1] *= al1;
-        acc[nt][mt][2] *= al0;
-        acc[nt][mt][3] *= al1;
+        for (int mt = 0; mt < KS; ++mt) {
+          acc[nt][mt][0] *= al0;
+          acc[nt][mt][1] *= al1;
+          acc[nt][mt][2] *= al0;
+          acc[nt][mt][3] *= al1;
+        }
       }
       pf[nt][0] = movmatrix_trans(x0);  // (k = tok 2q, 2q+1 ; n = g = r)
       pf[nt][1] = movmatrix_trans(x1);  // (k = tok 2q+8, 2q+9)
@@ -476,14 +478,17 @@ __global__ void __launch_bounds__(Cfg<KV, QT, D, NT, KIND, OCC>::kThreads, Cfg<K
   const int Hq = p.num_kv_heads * G;
   const int PT = p.partition_tokens;
 
+  // This grid covers tokens [start, start + span) of the sequence: all of it for plain decode, the
+  // part after the shared prefix for cascade decode.
   const int ctx = p.context_lens[s];
-  int ctx_eff = min(ctx, p.max_blocks * 16);
-  ctx_eff = min(ctx_eff, p.num_partitions * PT);
-  if (ctx_eff < ctx || ctx < 0) {
+  const int start = p.start_tokens;
+  const int ctx_cap = min(ctx, p.max_blocks * 16);
+  int span = min(max(ctx_cap - start, 0), p.num_partitions * PT);
+  if (ctx_cap < ctx || ctx < 0 || span < ctx_cap - start) {
     if (part == 0 && hk == 0 && threadIdx.x == 0) atomicOr(p.err, 8u);
-    ctx_eff = max(ctx_eff, 0);
   }
-  const int nparts = (ctx_eff + PT - 1) / PT;
+  const int ctx_eff = start + span;  // tokens [0, ctx_eff) exist for this grid's bookkeeping
+  const int nparts = (span + PT - 1) / PT;
   if (part >= max(nparts, 1)) return;
 
   // pa_decode_step: the CTA holding the sequence's last partition writes head hk's new K/V row
@@ -491,7 +496,9 @@ __global__ void __launch_bounds__(Cfg<KV, QT, D, NT, KIND, OCC>::kThreads, Cfg<K
   // page, and the proxy fence + barrier order the writes before this CTA's TMA loads.
   if (p.new_k != nullptr && part == max(nparts, 1) - 1) {
     const int64_t slot = p.new_slots[s];
-    if (slot >= 0 && slot < static_cast<int64_t>(p.num_blocks) * 16) {
+    // With a shared prefix the new token must lie past it (prefix blocks are read-only here).
+    const bool writable = start == 0 || nparts > 0;
+    if (writable && slot >= 0 && slot < static_cast<int64_t>(p.num_blocks) * 16) {
       constexpr int kChunks = D / 8;  // 16-byte input chunks per row
       for (int c = threadIdx.x; c < 2 * kChunks; c += C::kThreads) {
         const bool is_v = c >= kChunks;
@@ -524,7 +531,35 @@ __global__ void __launch_bounds__(Cfg<KV, QT, D, NT, KIND, OCC>::kThreads, Cfg<K
   }
 
   typedef uint16_t out_t;
-  if (ctx_eff == 0) {  // empty context: output 0
+  if (span == 0 && p.merge_prefix_inline) {
+    // Nothing past the shared prefix: the output is the merge of the prefix partials alone.
+    for (int idx = threadIdx.x; idx < G * D; idx += C::kThreads) {
+      const int g = idx / D, d = idx % D, h = hk * G + g;
+      const int64_t row0 = (static_cast<int64_t>(s) * Hq + h) * p.ws_parts;
+      float M = -INFINITY;
+      for (int k = 0; k < p.part_offset; ++k) M = fmaxf(M, p.ws_ml[(row0 + k) * 2]);
+      float num = 0.f, den = 0.f;
+      if (M != -INFINITY) {
+        for (int k = 0; k < p.part_offset; ++k) {
+          const float f = ex2(p.ws_ml[(row0 + k) * 2] - M);
+          num = fmaf(f, p.ws_acc[(row0 + k) * D + d], num);
+          den = fmaf(f, p.ws_ml[(row0 + k) * 2 + 1], den);
+        }
+      }
+      const float o = den > 0.f ? num / den * p.v_scale : 0.f;
+      uint16_t bits;
+      if constexpr (C::kQBf16) {
+        bits = __bfloat16_as_ushort(__float2bfloat16_rn(o));
+      } else {
+        bits = __half_as_ushort(__float2half_rn(o));
+      }
+      static_cast<uint16_t*>(p.out)[s * p.o_stride_s + h * p.o_stride_h + d] = bits;
+    }
+    return;
+  }
+  if (span == 0) {
+    if (p.always_partials) return;  // the merge kernel covers this sequence from its other partials
+    // empty context: output 0
     for (int i = threadIdx.x; i < G * D; i += C::kThreads) {
       const int g = i / D, d = i % D;
       static_cast<out_t*>(p.out)[s * p.o_stride_s + (hk * G + g) * p.o_stride_h + d] = 0;
@@ -533,7 +568,7 @@ __global__ void __launch_bounds__(Cfg<KV, QT, D, NT, KIND, OCC>::kThreads, Cfg<K
   }
 
   const int pages_per_part = PT / 16;
-  const int j0 = part * pages_per_part;
+  const int j0 = start / 16 + part * pages_per_part;
   const int j1 = min(j0 + pages_per_part, (ctx_eff + 15) / 16);
   const int n_w = max(0, (j1 - j0 - warp + C::kWarps - 1) / C::kWarps);  // pages of this warp (<= 32)
 
@@ -658,7 +693,8 @@ __global__ void __launch_bounds__(Cfg<KV, QT, D, NT, KIND, OCC>::kThreads, Cfg<K
   __syncthreads();
   if (any_fail) return;
 
-  const bool direct = nparts <= 1;
+  const bool inline_merge = p.merge_prefix_inline && nparts <= 1;
+  const bool direct = (!p.always_partials && nparts <= 1) || inline_merge;
   for (int idx = threadIdx.x; idx < G * D; idx += C::kThreads) {
     const int g = idx / D, d = idx % D;
     float M = -INFINITY;
@@ -672,6 +708,21 @@ __global__ void __launch_bounds__(Cfg<KV, QT, D, NT, KIND, OCC>::kThreads, Cfg<K
       den = fmaf(f, lg[w * C::kGPad + g], den);
     }
     const int h = hk * G + g;
+    if (inline_merge) {
+      // Fold in the shared-prefix partials (slots 0 .. part_offset - 1), prefix first, then this CTA.
+      const int64_t row0 = (static_cast<int64_t>(s) * Hq + h) * p.ws_parts;
+      float Mp = M;
+      for (int k = 0; k < p.part_offset; ++k) Mp = fmaxf(Mp, p.ws_ml[(row0 + k) * 2]);
+      float n2 = 0.f, d2 = 0.f;
+      for (int k = 0; k < p.part_offset; ++k) {
+        const float f = ex2(p.ws_ml[(row0 + k) * 2] - Mp);
+        n2 = fmaf(f, p.ws_acc[(row0 + k) * D + d], n2);
+        d2 = fmaf(f, p.ws_ml[(row0 + k) * 2 + 1], d2);
+      }
+      const float f = ex2(M - Mp);
+      num = fmaf(f, num, n2);
+      den = fmaf(f, den, d2);
+    }
     if (direct) {
       const float o = num / den * p.v_scale;
       out_t bits;
@@ -682,7 +733,7 @@ __global__ void __launch_bounds__(Cfg<KV, QT, D, NT, KIND, OCC>::kThreads, Cfg<K
       }
       static_cast<out_t*>(p.out)[s * p.o_stride_s + h * p.o_stride_h + d] = bits;
     } else {
-      const int64_t row = (static_cast<int64_t>(s) * Hq + h) * p.num_partitions + part;
+      const int64_t row = (static_cast<int64_t>(s) * Hq + h) * p.ws_parts + p.part_offset + part;
       p.ws_acc[row * D + d] = num;
       if (d == 0) {
         p.ws_ml[row * 2] = M;
@@ -700,13 +751,17 @@ __global__ void __launch_bounds__(D) reduce_kernel(const DecodeParams p) {
   pdl_launch_dependents();
   const int Hq = p.num_kv_heads * p.group;
   const int PT = p.partition_tokens;
-  int ctx_eff = min(p.context_lens[s], p.max_blocks * 16);
-  ctx_eff = max(0, min(ctx_eff, p.num_partitions * PT));
-  const int np = (ctx_eff + PT - 1) / PT;
-  if (np <= 1) return;  // the decode kernel wrote this row
-  const int64_t row0 = (static_cast<int64_t>(s) * Hq + h) * p.num_partitions;
+  const int ctx_cap = min(p.context_lens[s], p.max_blocks * 16);
+  const int span = min(max(ctx_cap - p.start_tokens, 0), p.num_partitions * PT);
+  const int np = p.part_offset + (span + PT - 1) / PT;
+  if (!p.always_partials && np <= 1) return;  // the decode kernel wrote this row
+  const int64_t row0 = (static_cast<int64_t>(s) * Hq + h) * p.ws_parts;
   float M = -INFINITY;
   for (int k = 0; k < np; ++k) M = fmaxf(M, p.ws_ml[(row0 + k) * 2]);
+  if (M == -INFINITY) {  // no token at all (empty context)
+    static_cast<uint16_t*>(p.out)[s * p.o_stride_s + h * p.o_stride_h + d] = 0;
+    return;
+  }
   float num = 0.f, den = 0.f;
 #pragma unroll 4
   for (int k = 0; k < np; ++k) {

@@ -31,6 +31,16 @@ struct DecodeParams {
   float* ws_acc;             // [B, Hq, P, D] un-normalised partial outputs (split only)
   float* ws_ml;              // [B, Hq, P, 2] partial (running max in log2 units, sum) (split only)
   uint32_t* err;             // error word (never null)
+  // Cascade (shared-prefix) decode: this grid covers tokens [start_tokens, ctx) of each sequence and
+  // always writes partials, at workspace slots part_offset + partition of rows ws_parts slots long.
+  // Plain decode: start_tokens 0, part_offset 0, ws_parts = num_partitions, always_partials 0.
+  int32_t start_tokens;
+  int32_t part_offset;
+  int32_t ws_parts;
+  int32_t always_partials;
+  // Cascade with an unsplit suffix: the decode CTA merges the prefix partials (slots [0, part_offset))
+  // with its own result and writes the output; no merge kernel runs.
+  int32_t merge_prefix_inline;
   // Fused new-token write (pa_decode_step); new_k == nullptr for plain pa_decode.
   const void* new_k;         // [B, Hkv, D] f16/bf16
   const void* new_v;
@@ -77,6 +87,28 @@ struct CacheParams {
 
 // src: 0 = f16, 1 = bf16 source; cache: KvType.
 cudaError_t launch_reshape_and_cache(int src_bf16, KvType cache, const CacheParams& p, cudaStream_t stream);
+
+// Shared-prefix attention (cascade.cu): query rows (sequence, query head) of every sequence against
+// the first prefix_tokens tokens, which every block-table row maps to the same blocks.
+struct PrefixParams {
+  const void* q;
+  int64_t q_stride_s, q_stride_h;
+  const int32_t* block_tables;
+  int64_t bt_stride;
+  const int32_t* context_lens;
+  int32_t num_seqs, num_blocks, num_kv_heads, group;
+  int32_t prefix_tokens;  // multiple of 16
+  int32_t chunk_tokens;   // tokens per CTA (multiple of 16, <= 512)
+  int32_t num_chunks;
+  float score_scale_log2;
+  float* ws_acc;
+  float* ws_ml;
+  int32_t ws_parts;
+  uint32_t* err;
+};
+constexpr int kPrefixChunkTokens = 256;
+cudaError_t launch_prefix(KvType kv, int head_dim, const CUtensorMap& k_map, const CUtensorMap& v_map,
+                          const PrefixParams& p, cudaStream_t stream);
 
 struct CopyParams {
   void* k_cache;

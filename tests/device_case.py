@@ -124,6 +124,20 @@ class DeviceCase:
                           kernel=kernel)
         return out
 
+    def cascade(self, fused: bool = True, partition_tokens: int = 0, out: Optional[torch.Tensor] = None,
+                error_word: Optional[torch.Tensor] = None) -> torch.Tensor:
+        """pa_decode_cascade over the workload's shared prefix (with the new-token write if fused)."""
+        w = self.w
+        out = self.out if out is None else out
+        n = pa.pa_decode_cascade_workspace_bytes(w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim, self.max_ctx,
+                                                 w.shared_prefix_tokens, partition_tokens)
+        ws = torch.empty(n, dtype=torch.uint8, device=self.device)
+        nk = (self.new_k, self.new_v, self.new_slots) if fused else (None, None, None)
+        pa.pa_decode_cascade(out, self.q, *nk, self.k_cache, self.v_cache, self.bt, self.lens,
+                             w.shared_prefix_tokens, w.scale, w.num_kv_heads, max_context_len=self.max_ctx,
+                             partition_tokens=partition_tokens, workspace=ws, error_word=error_word)
+        return out
+
     def pool_bytes(self):
         """(k, v) pools as host uint8 [NB, Hkv, 16, D * elem]."""
         w = self.w
