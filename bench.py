@@ -51,7 +51,7 @@ def parse():
                     help="fused: pa_decode_step (new-token write inside the decode launch); "
                          "separate: pa_reshape_and_cache then pa_decode; "
                          "cascade: pa_decode_cascade over the workload's shared prefix (prefix_gqa)")
-    ap.add_argument("--op", choices=["step", "copy_blocks", "kv_utilization"], default="step",
+    ap.add_argument("--op", choices=["step", "copy_blocks", "kv_utilization", "prefill"], default="step",
                     help="step: the decode step (the headline); copy_blocks: copy-on-write block copies; "
                          "kv_utilization: KV memory utilisation of the block allocator (host only)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -504,6 +504,62 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def run_prefill(args, rank, world, local_rank):
+    """Chunked-prefill attention: 8 sequences x 2048-token prompts, Llama-3-8B heads (32/8, D=128), bf16."""
+    import paged_kv_cache_385_b200 as pa
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    B, n, Hq, Hkv, D = 8, 2048, 32, 8, 128
+    nb = B * n // 16 + 64
+    g = torch.Generator(device=device)
+    g.manual_seed(77)
+    alloc = pa.BlockAllocator(nb, torch.randperm(nb, generator=torch.Generator().manual_seed(77)).tolist())
+    bt = pa.build_block_tables(alloc, [n] * B, n // 16)
+    kc = torch.randn(nb, Hkv, 16, D, generator=g, device=device).to(torch.bfloat16)
+    vc = torch.randn(nb, Hkv, 16, D, generator=g, device=device).to(torch.bfloat16)
+    q = torch.randn(B * n, Hq, D, generator=g, device=device).to(torch.bfloat16)
+    out = torch.empty_like(q)
+    qs = torch.arange(0, B * n + 1, n, dtype=torch.int32, device=device)
+    lens = torch.full((B,), n, dtype=torch.int32, device=device)
+    btd = bt.to(device)
+    # Causal FLOPs: QK^T and PV, 2 flops per MAC, position i sees i + 1 keys.
+    flops = B * Hq * 2 * 2 * D * (n * (n + 1) // 2)
+    K, Wm = max(5, args.steps // 100), max(3, args.warmup)
+
+    def call():
+        pa.pa_prefill(out, q, kc, vc, btd, qs, lens, n, D ** -0.5, Hkv)
+
+    for _ in range(Wm):
+        call()
+    torch.cuda.synchronize(device)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clocks:
+        a.record()
+        for _ in range(K):
+            call()
+        b.record()
+        torch.cuda.synchronize(device)
+    ms = a.elapsed_time(b) / K
+    tflops = flops / (ms / 1e3) / 1e12
+    peak_path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(peak_path) as f:
+            peak, src = float(json.load(f)["bf16_tflops"]), "measured (MEASURED_PEAKS.json bf16_tflops, cuBLAS burst)"
+    except Exception:
+        peak, src = 1590.0, "fallback"
+    if rank == 0:
+        print(json.dumps({
+            "metric": "chunked prefill attention over paged KV: TFLOP/s (causal, QK^T + PV)", "value": round(tflops, 1),
+            "unit": "TFLOP/s", "n_gpus": 1, "steps": K, "warmup": Wm, "ms_per_step": round(ms, 4),
+            "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+            "config": {"num_seqs": B, "prompt_tokens": n, "num_q_heads": Hq, "num_kv_heads": Hkv, "head_dim": D,
+                       "flops_per_call": flops},
+            "roofline": {"bound": "tensor", "achieved": round(tflops, 1), "peak": peak, "unit": "TFLOP/s",
+                         "frac": round(tflops / peak, 4), "traffic": None, "peak_source": src,
+                         "note": "warp-level mma.sync m16n8k16; the peak is a tcgen05 cuBLAS figure"},
+            "gpu_launches": K, "clocks": clocks.summary()}), flush=True)
+
+
 def run_copy_blocks(args, rank, world, local_rank):
     """Throughput of pa_copy_blocks on the workload's pool: 1024 distinct (src, dst) block pairs per call."""
     import paged_kv_cache_385_b200 as pa
@@ -608,6 +664,9 @@ def main():
         return 0
     if args.op == "copy_blocks":
         run_copy_blocks(args, rank, world, local_rank)
+        return 0
+    if args.op == "prefill":
+        run_prefill(args, rank, world, local_rank)
         return 0
     if args.impl == "reference":
         run_reference(args, rank, world)

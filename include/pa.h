@@ -195,6 +195,28 @@ size_t pa_decode_cascade_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, 
                                          int32_t head_dim, int32_t max_context_len, int32_t shared_prefix_tokens,
                                          int32_t partition_tokens);
 
+/*
+ * pa_prefill -- causal attention of a chunk of new tokens per sequence over its paged context
+ * (prompt prefill, or one chunk of a chunked prefill).
+ *   out, q        [T, Hq, D] device F16/BF16 (the caches' dtype), last stride 1, 16-B aligned rows. Rows
+ *                 query_start[s] .. query_start[s + 1] - 1 belong to sequence s: its last
+ *                 n_s = query_start[s + 1] - query_start[s] tokens.
+ *   k_cache, v_cache  [num_blocks, Hkv, 16, D] F16/BF16, holding every token of the context already
+ *                 (write the chunk's K/V with pa_reshape_and_cache first).
+ *   block_tables  [B, max_blocks] I32; query_start [B + 1] I32; context_lens [B] I32: tokens of
+ *                 sequence s including the chunk (n_s <= context_lens[s] <= 16 * max_blocks).
+ *   max_query_len host-known bound on n_s (sizes the grid without a device read).
+ * Row i of sequence s is position p = context_lens[s] - n_s + i and sees positions 0 .. p:
+ * out = softmax(scale * q K[0..p]^T) V[0..p], float32 accumulation, rounded to nearest even.
+ * Violations only the device can see (n_s > context_lens[s], n_s > max_query_len) set
+ * PA_DEVERR_CTX_RANGE. D in {64, 128}.
+ * Source: the notes page's kernels section (FlashAttention adapted to paged KV) and "vLLM 前世今生"
+ * section 5.4 (chunked prefill).
+ */
+int pa_prefill(pa_tensor* out, const pa_tensor* q, const pa_tensor* k_cache, const pa_tensor* v_cache,
+               const pa_tensor* block_tables, const pa_tensor* query_start, const pa_tensor* context_lens,
+               int32_t max_query_len, float scale, int32_t num_kv_heads, void* stream);
+
 /* Partition size pa_decode uses when opts->partition_tokens == 0 and a workspace is given
  * (0 = no split: the batch's B * Hkv (sequence, KV head) units already fill the GPU and every
  * context fits one CTA, <= 2048 tokens). Otherwise the largest of 2048, 1024, 512 that still gives

@@ -93,3 +93,33 @@ def decode_logical_one(q_vec: np.ndarray, k_seq: np.ndarray, v_seq: np.ndarray, 
     """One (sequence, query head) output from the logical rows: what sampled full-size checks call."""
     hk = q_head // (num_q_heads // num_kv_heads)
     return attend(q_vec, k_seq[:, hk, :], v_seq[:, hk, :], scale)
+
+
+def prefill_paged(q: np.ndarray, k_pool: np.ndarray, v_pool: np.ndarray, block_tables: np.ndarray,
+                  query_start: Sequence[int], context_lens: Sequence[int], scale: float, num_kv_heads: int,
+                  kv_dtype: str, block_size: int = 16) -> np.ndarray:
+    """Causal attention of a chunk of new tokens per sequence over its paged context (float64).
+
+    Sequence s owns query rows query_start[s] .. query_start[s + 1] - 1, the last
+    n_s = query_start[s + 1] - query_start[s] tokens of its context_lens[s] tokens (all already
+    written to the pool). Row i of the chunk is position p = context_lens[s] - n_s + i and attends
+    over positions 0 .. p (itself included): out = softmax(scale * q K[0..p]^T) V[0..p].
+    Source: the notes page's kernels section (attention over paged KV, FlashAttention adapted to
+    paging) and "vLLM 前世今生" §5.4 (chunked prefill: a long prompt's prefill split into chunks).
+    """
+    q = np.asarray(q, dtype=np.float64)
+    T, Hq, D = q.shape
+    G = Hq // num_kv_heads
+    out = np.zeros((T, Hq, D), dtype=np.float64)
+    for s in range(len(context_lens)):
+        r0, r1 = int(query_start[s]), int(query_start[s + 1])
+        n = int(context_lens[s])
+        start = n - (r1 - r0)
+        for hk in range(num_kv_heads):
+            K = gather_context(k_pool, block_tables[s], n, hk, kv_dtype, 1.0, block_size)
+            V = gather_context(v_pool, block_tables[s], n, hk, kv_dtype, 1.0, block_size)
+            for i in range(r1 - r0):
+                p = start + i
+                for h in range(hk * G, (hk + 1) * G):
+                    out[r0 + i, h] = attend(q[r0 + i, h], K[:p + 1], V[:p + 1], scale)
+    return out

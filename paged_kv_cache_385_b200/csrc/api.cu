@@ -471,7 +471,7 @@ static int decode_impl(pa_tensor* out, const pa_tensor* q, const pa_tensor* k_ca
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e;
   if (cascade) {
-    pa::PrefixParams pp{};
+    pa::MqParams pp{};
     pp.q = q->data;
     pp.q_stride_s = q->stride[0];
     pp.q_stride_h = q->stride[1];
@@ -482,6 +482,7 @@ static int decode_impl(pa_tensor* out, const pa_tensor* q, const pa_tensor* k_ca
     pp.num_blocks = p.num_blocks;
     pp.num_kv_heads = num_kv_heads;
     pp.group = p.group;
+    pp.max_blocks = p.max_blocks;
     pp.prefix_tokens = prefix_tokens;
     pp.chunk_tokens = pa::kPrefixChunkTokens;
     pp.num_chunks = static_cast<int32_t>(n_pre);
@@ -567,6 +568,75 @@ size_t pa_decode_cascade_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, 
   }
   const int64_t P = std::max<int64_t>(1, (span + pt - 1) / pt);
   return workspace_layout(num_seqs, num_q_heads, head_dim, n_pre + P, nullptr);
+}
+
+int pa_prefill(pa_tensor* out, const pa_tensor* q, const pa_tensor* k_cache, const pa_tensor* v_cache,
+               const pa_tensor* block_tables, const pa_tensor* query_start, const pa_tensor* context_lens,
+               int32_t max_query_len, float scale, int32_t num_kv_heads, void* stream) {
+  int st;
+  if ((st = check_tensor(out, "out", 3)) || (st = check_tensor(q, "q", 3)) || (st = check_tensor(k_cache, "k_cache", 4)) ||
+      (st = check_tensor(v_cache, "v_cache", 4)) || (st = check_tensor(block_tables, "block_tables", 2)) ||
+      (st = check_tensor(query_start, "query_start", 1)) || (st = check_tensor(context_lens, "context_lens", 1)))
+    return st;
+  const int64_t T = q->shape[0], Hq = q->shape[1], D = q->shape[2], B = block_tables->shape[0];
+  const int cd = k_cache->dtype;
+  if (cd != PA_F16 && cd != PA_BF16) return fail(PA_ERR_UNSUPPORTED, "prefill takes F16 or BF16 caches");
+  if (q->dtype != cd || out->dtype != cd || v_cache->dtype != cd)
+    return fail(PA_ERR_INVALID_ARG, "q, out and both caches must have one dtype");
+  for (int i = 0; i < 3; ++i)
+    if (out->shape[i] != q->shape[i]) return fail(PA_ERR_INVALID_ARG, "out shape differs from q shape");
+  for (int i = 0; i < 4; ++i)
+    if (v_cache->shape[i] != k_cache->shape[i]) return fail(PA_ERR_INVALID_ARG, "v_cache shape differs from k_cache");
+  if (num_kv_heads <= 0 || k_cache->shape[1] != num_kv_heads || Hq % num_kv_heads)
+    return fail(PA_ERR_INVALID_ARG, "num_kv_heads must equal k_cache.shape[1] and divide num_q_heads");
+  if (k_cache->shape[2] != PA_BLOCK_SIZE || k_cache->shape[3] != D)
+    return fail(PA_ERR_INVALID_ARG, "cache shape must be [num_blocks, Hkv, 16, %lld]", (long long)D);
+  if (D != 64 && D != 128) return fail(PA_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
+  if (!is_contiguous(k_cache) || !is_contiguous(v_cache)) return fail(PA_ERR_INVALID_ARG, "caches must be contiguous");
+  if (block_tables->dtype != PA_I32 || (block_tables->stride[1] != 1 && block_tables->shape[1] > 1))
+    return fail(PA_ERR_INVALID_ARG, "block_tables must be I32 [num_seqs, max_blocks], last stride 1");
+  if (query_start->dtype != PA_I32 || query_start->shape[0] != B + 1 || (query_start->stride[0] != 1 && B > 0))
+    return fail(PA_ERR_INVALID_ARG, "query_start must be contiguous I32 [num_seqs + 1]");
+  if (context_lens->dtype != PA_I32 || context_lens->shape[0] != B || (context_lens->stride[0] != 1 && B > 1))
+    return fail(PA_ERR_INVALID_ARG, "context_lens must be contiguous I32 [num_seqs]");
+  if (!std::isfinite(scale)) return fail(PA_ERR_INVALID_ARG, "scale must be finite");
+  if (T == 0 || B == 0) return ok();
+  if (max_query_len <= 0) return fail(PA_ERR_INVALID_ARG, "max_query_len must be > 0");
+  if (B > 65535 || num_kv_heads > 65535) return fail(PA_ERR_UNSUPPORTED, "num_seqs and num_kv_heads must be <= 65535");
+  if (k_cache->shape[0] * num_kv_heads * 16 > 0x7fffffffLL) return fail(PA_ERR_UNSUPPORTED, "pool too large");
+  if (q->stride[2] != 1 || out->stride[2] != 1 || !aligned(q->data, 16) || !aligned(out->data, 16) ||
+      q->stride[0] % 8 || q->stride[1] % 8 || out->stride[0] % 8 || out->stride[1] % 8)
+    return fail(PA_ERR_INVALID_ARG, "q/out rows must be contiguous and 16-byte aligned");
+  if (!aligned(k_cache->data, 128) || !aligned(v_cache->data, 128))
+    return fail(PA_ERR_INVALID_ARG, "caches must be 128-byte aligned");
+  if (!out->data || !q->data || !k_cache->data || !v_cache->data || !block_tables->data || !query_start->data ||
+      !context_lens->data)
+    return fail(PA_ERR_INVALID_ARG, "NULL data pointer");
+  pa::MqParams p{};
+  p.q = q->data;
+  p.q_stride_s = q->stride[0];
+  p.q_stride_h = q->stride[1];
+  p.out = out->data;
+  p.o_stride_t = out->stride[0];
+  p.o_stride_h = out->stride[1];
+  p.block_tables = static_cast<const int32_t*>(block_tables->data);
+  p.bt_stride = block_tables->stride[0];
+  p.context_lens = static_cast<const int32_t*>(context_lens->data);
+  p.query_start = static_cast<const int32_t*>(query_start->data);
+  p.num_seqs = static_cast<int32_t>(B);
+  p.num_blocks = static_cast<int32_t>(k_cache->shape[0]);
+  p.num_kv_heads = num_kv_heads;
+  p.group = static_cast<int32_t>(Hq / num_kv_heads);
+  p.max_blocks = static_cast<int32_t>(std::min<int64_t>(block_tables->shape[1], 0x7fffffff / 16));
+  p.score_scale_log2 = scale * 1.4426950408889634f;
+  p.err = library_error_word();
+  if (!p.err) return fail(PA_ERR_CUDA, "no device error word (no current CUDA device?)");
+  CUtensorMap km, vm;
+  if ((st = encode_pool_map(&km, k_cache, 2)) || (st = encode_pool_map(&vm, v_cache, 2))) return st;
+  const pa::KvType kv = cd == PA_BF16 ? pa::KvType::BF16 : pa::KvType::F16;
+  cudaError_t e = pa::launch_prefill(kv, static_cast<int>(D), km, vm, p, max_query_len, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(PA_ERR_CUDA, "prefill launch: %s", cudaGetErrorString(e));
+  return ok();
 }
 
 int pa_decode_step(pa_tensor* out, const pa_tensor* q, const pa_tensor* key, const pa_tensor* value,

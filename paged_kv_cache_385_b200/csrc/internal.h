@@ -88,27 +88,34 @@ struct CacheParams {
 // src: 0 = f16, 1 = bf16 source; cache: KvType.
 cudaError_t launch_reshape_and_cache(int src_bf16, KvType cache, const CacheParams& p, cudaStream_t stream);
 
-// Shared-prefix attention (cascade.cu): query rows (sequence, query head) of every sequence against
-// the first prefix_tokens tokens, which every block-table row maps to the same blocks.
-struct PrefixParams {
+// Multi-query attention (multiquery.cu). Shared prefix: query rows (sequence, query head) of every
+// sequence against the first prefix_tokens tokens, which every block-table row maps to the same
+// blocks -> partials. Chunked prefill: rows (new token, query head) of each sequence, causal over
+// its pages -> out.
+struct MqParams {
   const void* q;
-  int64_t q_stride_s, q_stride_h;
+  int64_t q_stride_s, q_stride_h;  // prefix: per sequence; prefill: per token row of q
   const int32_t* block_tables;
   int64_t bt_stride;
   const int32_t* context_lens;
-  int32_t num_seqs, num_blocks, num_kv_heads, group;
-  int32_t prefix_tokens;  // multiple of 16
-  int32_t chunk_tokens;   // tokens per CTA (multiple of 16, <= 512)
+  int32_t num_seqs, num_blocks, num_kv_heads, group, max_blocks;
+  int32_t prefix_tokens;  // prefix: multiple of 16
+  int32_t chunk_tokens;   // prefix: tokens per CTA (multiple of 16)
   int32_t num_chunks;
   float score_scale_log2;
-  float* ws_acc;
+  float* ws_acc;  // prefix partials
   float* ws_ml;
   int32_t ws_parts;
+  const int32_t* query_start;  // prefill: [B + 1] rows of q per sequence
+  void* out;                   // prefill: [T, Hq, D]
+  int64_t o_stride_t, o_stride_h;
   uint32_t* err;
 };
 constexpr int kPrefixChunkTokens = 256;
 cudaError_t launch_prefix(KvType kv, int head_dim, const CUtensorMap& k_map, const CUtensorMap& v_map,
-                          const PrefixParams& p, cudaStream_t stream);
+                          const MqParams& p, cudaStream_t stream);
+cudaError_t launch_prefill(KvType kv, int head_dim, const CUtensorMap& k_map, const CUtensorMap& v_map,
+                           const MqParams& p, int max_query_len, cudaStream_t stream);
 
 struct CopyParams {
   void* k_cache;

@@ -1,20 +1,22 @@
-// Shared-prefix ("cascade") attention for sm_100a: the query rows of every sequence against the
-// pages of a prefix they all share, read once per KV head instead of once per sequence.
+// Multi-query paged attention for sm_100a: tiles of 16 query rows per warp against a stream of
+// 16-token pages, the dense tensor-core part of the path. Two uses:
 //
-// Source: "vLLM 前世今生" section 3.2 (several sequences point at the same physical blocks, e.g. a
-// shared prompt prefix) and the notes page's prefix-caching section (identical prompt prefixes are
-// computed once and reused). Attention over a shared prefix is then, per KV head, a dense
-// contraction of all B * G query rows with the prefix's keys and values: rows (s, g) ->
-// partial softmax state (m, l, acc) over the prefix tokens, merged later with each sequence's own
-// suffix by the partition-merge kernel. The result equals the plain definition over the whole
-// context (it is the same softmax split at a token boundary).
+// * Shared prefix ("cascade", MODE 0). Source: "vLLM 前世今生" section 3.2 (several sequences point at
+//   the same physical blocks, e.g. a shared prompt prefix) and the notes page's prefix-caching
+//   section (a shared prompt prefix computed once). Per KV head, all B * G query rows (sequence s,
+//   group member g) against the prefix pages every block table shares: partial softmax state
+//   (m, l, acc) per row and prefix chunk, merged later with the sequence's own suffix. It equals the
+//   plain definition over the whole context (the same softmax split at a token boundary).
+// * Chunked prefill (MODE 1). Source: the notes page's kernels section (FlashAttention adapted to
+//   paged KV) and "vLLM 前世今生" section 5.4 (chunked prefill). Per sequence and KV head, rows
+//   (new token i, group member g) attend causally over the sequence's pages: position
+//   start + i sees tokens 0 .. start + i. Output written directly.
 //
-// Kernel: grid (row tiles of 64 query rows, KV head, prefix chunk). Four consumer warps own 16 rows
-// each; a fifth warp produces: it streams the chunk's K and V pages (taken from sequence 0's block
-// table; every sequence's table must hold the same prefix blocks, which the consumers check) with
-// TMA into a ring of stages guarded by full/empty mbarriers. Per 16-token page a consumer warp does
-// S[16 rows x 16 tok] = Q K^T (mma.sync m16n8k16, K^T fragments by ldmatrix), an online softmax per
-// row, and O[16 x D] += P V (P reused from the score fragments, V^T fragments by ldmatrix.trans).
+// Kernel: four consumer warps own 16 rows each; a fifth warp produces: it streams the CTA's K and V
+// pages with TMA into a ring of stages guarded by full/empty mbarriers. Per page a consumer warp
+// does S[16 rows x 16 tok] = Q K^T (mma.sync m16n8k16, K^T fragments by ldmatrix), an online
+// softmax per row (per-row token limits: context, prefix end, or the causal diagonal), and
+// O[16 x D] += P V (P reused from the score fragments, V^T fragments by ldmatrix.trans).
 #include "internal.h"
 #include "pa_device.cuh"
 
@@ -42,26 +44,53 @@ __device__ __forceinline__ uint32_t swz128(int tok, int chunk) {
   return static_cast<uint32_t>(tok * 128 + ((chunk ^ (tok & 7)) << 4));
 }
 
-template <KvType KV, int D>
-__global__ void __launch_bounds__(PCfg<KV, D>::kThreads) prefix_kernel(const __grid_constant__ CUtensorMap kmap,
-                                                                        const __grid_constant__ CUtensorMap vmap,
-                                                                        const PrefixParams p) {
+template <KvType KV, int D, int MODE>
+__global__ void __launch_bounds__(PCfg<KV, D>::kThreads) mq_kernel(const __grid_constant__ CUtensorMap kmap,
+                                                                    const __grid_constant__ CUtensorMap vmap,
+                                                                    const MqParams p) {
   using C = PCfg<KV, D>;
+  constexpr bool kPrefill = MODE == 1;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t ring = smem_u32(smem);
   const uint32_t full0 = smem_u32(smem + kPrefixStages * C::kStageBytes);
   const uint32_t empty0 = full0 + 8 * kPrefixStages;
 
-  const int tile = blockIdx.x, hk = blockIdx.y, chunk = blockIdx.z;
+  const int tile = blockIdx.x, hk = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = p.group;
   const int Hq = p.num_kv_heads * G;
-  const int num_rows = p.num_seqs * G;
   pdl_wait();
 
-  const int j0 = chunk * (p.chunk_tokens / 16);
-  const int npages = min(p.chunk_tokens / 16, p.prefix_tokens / 16 - j0);
+  // Rows and pages of this CTA.
+  int chunk = 0, s_seq = 0, num_rows, j0, npages, q_row0 = 0, start = 0;
+  const int32_t* bt_row;
+  if constexpr (kPrefill) {
+    s_seq = blockIdx.z;
+    q_row0 = p.query_start[s_seq];
+    const int n_new = p.query_start[s_seq + 1] - q_row0;
+    num_rows = n_new * G;
+    if (tile * kRowsPerCta >= num_rows) return;
+    const int ctx = p.context_lens[s_seq];
+    start = ctx - n_new;
+    if (tile == 0 && threadIdx.x == 0 && num_rows > static_cast<int>(gridDim.x) * kRowsPerCta)
+      atomicOr(p.err, 8u);  // more new tokens than max_query_len: the rows past the grid are not computed
+    const int last_tok = min(tile * kRowsPerCta + kRowsPerCta, num_rows) - 1;
+    const int last_key = start + last_tok / G;  // the CTA's last row sees keys 0 .. last_key
+    if (start < 0 || ctx > p.max_blocks * 16) {
+      if (threadIdx.x == 0) atomicOr(p.err, 8u);
+      return;
+    }
+    j0 = 0;
+    npages = last_key / 16 + 1;
+    bt_row = p.block_tables + static_cast<int64_t>(s_seq) * p.bt_stride;
+  } else {
+    chunk = blockIdx.z;
+    num_rows = p.num_seqs * G;
+    j0 = chunk * (p.chunk_tokens / 16);
+    npages = min(p.chunk_tokens / 16, p.prefix_tokens / 16 - j0);
+    bt_row = p.block_tables;  // sequence 0's row: every row shares these blocks
+  }
 
   if (threadIdx.x == 0) {
     for (int st = 0; st < kPrefixStages; ++st) {
@@ -75,13 +104,15 @@ __global__ void __launch_bounds__(PCfg<KV, D>::kThreads) prefix_kernel(const __g
   const uint64_t deadline = globaltimer_ns() + 2000000000ull;
   bool ok = true;
   if (warp == kConsumerWarps) {
-    // ---- producer: block ids in lanes, lane 0 streams the pages -------------------------------
+    // ---- producer: block ids 32 at a time in lanes, lane 0 streams the pages ------------------
     int bid = -1;
-    if (lane < npages) bid = p.block_tables[j0 + lane];  // sequence 0's row
-    const bool bad = lane < npages && (bid < 0 || bid >= p.num_blocks);
-    if (__any_sync(kFull, bad) && lane == 0) atomicOr(p.err, 1u);
     if (lane == 0) prefetch_tensormap(&kmap), prefetch_tensormap(&vmap);
     for (int i = 0; i < npages; ++i) {
+      if ((i & 31) == 0) {
+        bid = i + lane < npages ? bt_row[j0 + i + lane] : -1;
+        const bool bad = i + lane < npages && (bid < 0 || bid >= p.num_blocks);
+        if (__any_sync(kFull, bad) && lane == 0) atomicOr(p.err, 1u);
+      }
       const int b = __shfl_sync(kFull, bid, i & 31);
       const int st = i % kPrefixStages;
       if (lane == 0 && ok) {
@@ -116,23 +147,24 @@ __global__ void __launch_bounds__(PCfg<KV, D>::kThreads) prefix_kernel(const __g
   const int r = lane >> 2, q4 = lane & 3;
   const int row_lo = tile * kRowsPerCta + warp * 16 + r, row_hi = row_lo + 8;
 
-  // Rows are (sequence, query head in the group); a row's tokens are limited by its context.
+  // A row's last visible token + 1: its context, the prefix end, or its causal diagonal.
   auto row_limit = [&](int row) {
     if (row >= num_rows) return 0;
+    if constexpr (kPrefill) return start + row / G + 1;
     return min(p.context_lens[row / G], p.prefix_tokens);
   };
   const int lim_lo = row_limit(row_lo), lim_hi = row_limit(row_hi);
   int lim_max = max(lim_lo, lim_hi);
   for (int off = 4; off < 32; off <<= 1) lim_max = max(lim_max, __shfl_xor_sync(kFull, lim_max, off));
 
-  // Every sequence of these rows must map the prefix pages of this chunk to sequence 0's blocks.
-  {
+  if constexpr (!kPrefill) {
+    // Every sequence of these rows must map the prefix pages of this chunk to sequence 0's blocks.
     const int s_first = min(tile * kRowsPerCta + warp * 16, num_rows - 1) / G;
     const int s_last = min(tile * kRowsPerCta + warp * 16 + 15, num_rows - 1) / G;
     bool mismatch = false;
     for (int idx = lane; idx < (s_last - s_first + 1) * npages; idx += 32) {
-      const int s = s_first + idx / npages, j = j0 + idx % npages;
-      mismatch |= p.block_tables[s * p.bt_stride + j] != p.block_tables[j];
+      const int sq = s_first + idx / npages, j = j0 + idx % npages;
+      mismatch |= p.block_tables[sq * p.bt_stride + j] != p.block_tables[j];
     }
     if (__any_sync(kFull, mismatch) && lane == 0) atomicOr(p.err, 16u);
   }
@@ -141,8 +173,8 @@ __global__ void __launch_bounds__(PCfg<KV, D>::kThreads) prefix_kernel(const __g
   {
     auto qrow = [&](int row) -> const uint16_t* {
       const int rr = min(row, num_rows - 1);
-      return static_cast<const uint16_t*>(p.q) + static_cast<int64_t>(rr / G) * p.q_stride_s +
-             static_cast<int64_t>(hk * G + rr % G) * p.q_stride_h;
+      const int64_t qr = kPrefill ? static_cast<int64_t>(q_row0 + rr / G) : static_cast<int64_t>(rr / G);
+      return static_cast<const uint16_t*>(p.q) + qr * p.q_stride_s + static_cast<int64_t>(hk * G + rr % G) * p.q_stride_h;
     };
     const uint16_t* ql = qrow(row_lo);
     const uint16_t* qh = qrow(row_hi);
@@ -176,6 +208,11 @@ __global__ void __launch_bounds__(PCfg<KV, D>::kThreads) prefix_kernel(const __g
     }
     const uint32_t kb = ring + st * C::kStageBytes, vb = kb + C::kPageBytes;
     const int t0 = (j0 + i) * 16;
+    if (t0 >= lim_max) {  // past every row of this warp (causal tail): release the stage only
+      __syncwarp();
+      if (lane == 0) mbar_arrive(empty0 + 8 * st);
+      continue;
+    }
 
     // S = Q K^T for tokens t0 .. t0 + 15 (two n-tiles of 8 tokens).
     float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
@@ -260,20 +297,36 @@ __global__ void __launch_bounds__(PCfg<KV, D>::kThreads) prefix_kernel(const __g
   l_hi += __shfl_xor_sync(kFull, l_hi, 1);
   l_hi += __shfl_xor_sync(kFull, l_hi, 2);
 
-  // Partial state of each row -> workspace slot `chunk` of (sequence, query head).
+  if constexpr (kPrefill) {
+    // Normalised rows straight to the output.
 #pragma unroll
-  for (int half = 0; half < 2; ++half) {
-    const int row = half ? row_hi : row_lo;
-    if (row >= num_rows) continue;
-    const int s = row / G, h = hk * G + row % G;
-    const int64_t slot = (static_cast<int64_t>(s) * Hq + h) * p.ws_parts + chunk;
-    float* dst = p.ws_acc + slot * D;
+    for (int half = 0; half < 2; ++half) {
+      const int row = half ? row_hi : row_lo;
+      if (row >= num_rows) continue;
+      const float inv = 1.f / (half ? l_hi : l_lo);
+      uint16_t* dst = static_cast<uint16_t*>(p.out) + static_cast<int64_t>(q_row0 + row / G) * p.o_stride_t +
+                      static_cast<int64_t>(hk * G + row % G) * p.o_stride_h;
 #pragma unroll
-    for (int n = 0; n < NT; ++n)
-      *reinterpret_cast<float2*>(dst + 8 * n + 2 * q4) = make_float2(acc[n][2 * half], acc[n][2 * half + 1]);
-    if (q4 == 0) {
-      p.ws_ml[slot * 2] = half ? m_hi : m_lo;
-      p.ws_ml[slot * 2 + 1] = half ? l_hi : l_lo;
+      for (int n = 0; n < NT; ++n)
+        *reinterpret_cast<uint32_t*>(dst + 8 * n + 2 * q4) =
+            pack2<C::kBf16>(acc[n][2 * half] * inv, acc[n][2 * half + 1] * inv);
+    }
+  } else {
+    // Partial state of each row -> workspace slot `chunk` of (sequence, query head).
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const int row = half ? row_hi : row_lo;
+      if (row >= num_rows) continue;
+      const int sq = row / G, h = hk * G + row % G;
+      const int64_t slot = (static_cast<int64_t>(sq) * Hq + h) * p.ws_parts + chunk;
+      float* dst = p.ws_acc + slot * D;
+#pragma unroll
+      for (int n = 0; n < NT; ++n)
+        *reinterpret_cast<float2*>(dst + 8 * n + 2 * q4) = make_float2(acc[n][2 * half], acc[n][2 * half + 1]);
+      if (q4 == 0) {
+        p.ws_ml[slot * 2] = half ? m_hi : m_lo;
+        p.ws_ml[slot * 2 + 1] = half ? l_hi : l_lo;
+      }
     }
   }
 }
@@ -294,30 +347,43 @@ cudaError_t launch_pdl_prefix(void (*kern)(KArgs...), dim3 grid, dim3 block, siz
   return cudaLaunchKernelEx(&cfg, kern, args...);
 }
 
-template <KvType KV, int D>
-cudaError_t launch_prefix_t(const CUtensorMap& km, const CUtensorMap& vm, const PrefixParams& p, cudaStream_t st) {
+template <KvType KV, int D, int MODE>
+cudaError_t launch_mq_t(const CUtensorMap& km, const CUtensorMap& vm, const MqParams& p, dim3 grid, cudaStream_t st) {
   using C = PCfg<KV, D>;
-  auto kern = prefix_kernel<KV, D>;
+  auto kern = mq_kernel<KV, D, MODE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
-  const int rows = p.num_seqs * p.group;
-  const dim3 grid((rows + kRowsPerCta - 1) / kRowsPerCta, p.num_kv_heads, p.num_chunks);
   return launch_pdl_prefix(kern, grid, dim3(C::kThreads), C::kSmemBytes, st, km, vm, p);
+}
+
+template <int MODE>
+cudaError_t launch_mq(KvType kv, int head_dim, const CUtensorMap& km, const CUtensorMap& vm, const MqParams& p,
+                      dim3 grid, cudaStream_t st) {
+  if (kv == KvType::F16) {
+    return head_dim == 128 ? launch_mq_t<KvType::F16, 128, MODE>(km, vm, p, grid, st)
+                           : launch_mq_t<KvType::F16, 64, MODE>(km, vm, p, grid, st);
+  }
+  if (kv == KvType::BF16) {
+    return head_dim == 128 ? launch_mq_t<KvType::BF16, 128, MODE>(km, vm, p, grid, st)
+                           : launch_mq_t<KvType::BF16, 64, MODE>(km, vm, p, grid, st);
+  }
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace
 
-cudaError_t launch_prefix(KvType kv, int head_dim, const CUtensorMap& km, const CUtensorMap& vm, const PrefixParams& p,
+cudaError_t launch_prefix(KvType kv, int head_dim, const CUtensorMap& km, const CUtensorMap& vm, const MqParams& p,
                           cudaStream_t st) {
-  if (kv == KvType::F16) {
-    return head_dim == 128 ? launch_prefix_t<KvType::F16, 128>(km, vm, p, st)
-                           : launch_prefix_t<KvType::F16, 64>(km, vm, p, st);
-  }
-  if (kv == KvType::BF16) {
-    return head_dim == 128 ? launch_prefix_t<KvType::BF16, 128>(km, vm, p, st)
-                           : launch_prefix_t<KvType::BF16, 64>(km, vm, p, st);
-  }
-  return cudaErrorInvalidValue;
+  const int rows = p.num_seqs * p.group;
+  const dim3 grid((rows + kRowsPerCta - 1) / kRowsPerCta, p.num_kv_heads, p.num_chunks);
+  return launch_mq<0>(kv, head_dim, km, vm, p, grid, st);
+}
+
+cudaError_t launch_prefill(KvType kv, int head_dim, const CUtensorMap& km, const CUtensorMap& vm, const MqParams& p,
+                           int max_query_len, cudaStream_t st) {
+  const int64_t rows = static_cast<int64_t>(max_query_len) * p.group;
+  const dim3 grid(static_cast<unsigned>((rows + kRowsPerCta - 1) / kRowsPerCta), p.num_kv_heads, p.num_seqs);
+  return launch_mq<1>(kv, head_dim, km, vm, p, grid, st);
 }
 
 }  // namespace pa

@@ -1,0 +1,86 @@
+"""GPU parity of chunked prefill (pa_prefill) against the float64 oracle's causal definition."""
+import numpy as np
+import pytest
+import torch
+
+import paged_kv_cache_385_b200 as pa
+from oracle import attention
+from tests.device_case import TOL
+
+pytestmark = pytest.mark.gpu
+
+
+def _build(ctxs, news, hq, hkv, d, dtype, seed):
+    g = torch.Generator().manual_seed(seed)
+    B = len(ctxs)
+    nb = sum(-(-c // 16) for c in ctxs) + 11
+    order = torch.randperm(nb, generator=g).tolist()
+    alloc = pa.BlockAllocator(nb, order)
+    mb = max(-(-c // 16) for c in ctxs)
+    bt = pa.build_block_tables(alloc, ctxs, mb)
+    # Pools start as random bytes (NaN patterns included) so unwritten slots are never read.
+    kc = torch.randint(0, 256, (nb, hkv, 16, d * 2), generator=g, dtype=torch.uint8).view(dtype).view(nb, hkv, 16, d)
+    vc = torch.randint(0, 256, (nb, hkv, 16, d * 2), generator=g, dtype=torch.uint8).view(dtype).view(nb, hkv, 16, d)
+    K = [torch.randn(c, hkv, d, generator=g).to(dtype) for c in ctxs]
+    V = [torch.randn(c, hkv, d, generator=g).to(dtype) for c in ctxs]
+    seqs = [s for s in range(B) for _ in range(ctxs[s])]
+    poss = [p for s in range(B) for p in range(ctxs[s])]
+    kc, vc = kc.cuda(), vc.cuda()
+    pa.pa_reshape_and_cache(torch.cat(K).cuda(), torch.cat(V).cuda(), pa.pa_slots_for_positions(bt, seqs, poss).cuda(),
+                            kc, vc)
+    qs = torch.tensor([0] + np.cumsum(news).tolist(), dtype=torch.int32)
+    q = torch.randn(int(qs[-1]), hq, d, generator=g).to(dtype)
+    return bt, kc, vc, q, qs
+
+
+def _oracle(bt, kc, vc, q, qs, ctxs, scale, hkv, kvd):
+    shape = kc.shape
+    kb = kc.view(torch.uint8).reshape(shape[0], shape[1], 16, -1).cpu().numpy()
+    vb = vc.view(torch.uint8).reshape(shape[0], shape[1], 16, -1).cpu().numpy()
+    return attention.prefill_paged(q.double().numpy(), kb, vb, bt.numpy(), qs.tolist(), ctxs, scale, hkv, kvd)
+
+
+@pytest.mark.parametrize("ctxs,news,hq,hkv,d,dtype", [
+    ([37, 160, 90], [37, 16, 70], 8, 2, 128, torch.bfloat16),
+    ([1, 64, 200, 33], [1, 64, 5, 33], 4, 4, 64, torch.float16),
+    ([300, 129], [150, 129], 16, 2, 128, torch.float16),
+])
+def test_prefill_matches_oracle(ctxs, news, hq, hkv, d, dtype):
+    bt, kc, vc, q, qs = _build(ctxs, news, hq, hkv, d, dtype, seed=sum(ctxs))
+    out = torch.full((q.shape[0], hq, d), float("nan"), dtype=dtype, device="cuda")
+    pa.pa_prefill(out, q.cuda(), kc, vc, bt.cuda(), qs.cuda(), torch.tensor(ctxs, dtype=torch.int32).cuda(),
+                  max(news), 1.0 / np.sqrt(d), hkv)
+    torch.cuda.synchronize()
+    assert pa.pa_read_device_error(clear=True) == 0
+    want = _oracle(bt, kc, vc, q, qs, ctxs, 1.0 / np.sqrt(d), hkv, "bf16" if dtype == torch.bfloat16 else "f16")
+    err = float(np.max(np.abs(out.double().cpu().numpy() - want)))
+    assert err <= TOL["bf16" if dtype == torch.bfloat16 else "f16"], err
+
+
+def test_chunked_equals_whole_and_last_row_equals_decode():
+    ctxs, hq, hkv, d = [100], 8, 2, 128
+    bt, kc, vc, q, _ = _build(ctxs, [100], hq, hkv, d, torch.bfloat16, seed=5)
+    lens = torch.tensor(ctxs, dtype=torch.int32).cuda()
+    whole = torch.empty(100, hq, d, dtype=torch.bfloat16, device="cuda")
+    pa.pa_prefill(whole, q.cuda(), kc, vc, bt.cuda(), torch.tensor([0, 100], dtype=torch.int32).cuda(), lens, 100,
+                  0.09, hkv)
+    first = torch.empty(40, hq, d, dtype=torch.bfloat16, device="cuda")
+    second = torch.empty(60, hq, d, dtype=torch.bfloat16, device="cuda")
+    pa.pa_prefill(first, q[:40].cuda(), kc, vc, bt.cuda(), torch.tensor([0, 40], dtype=torch.int32).cuda(),
+                  torch.tensor([40], dtype=torch.int32).cuda(), 40, 0.09, hkv)
+    pa.pa_prefill(second, q[40:].cuda(), kc, vc, bt.cuda(), torch.tensor([0, 60], dtype=torch.int32).cuda(), lens, 60,
+                  0.09, hkv)
+    dec = torch.empty(1, hq, d, dtype=torch.bfloat16, device="cuda")
+    pa.pa_decode(dec, q[99:].cuda(), kc, vc, bt.cuda(), lens, 0.09, hkv)
+    torch.cuda.synchronize()
+    assert (whole.double() - torch.cat([first, second]).double()).abs().max().item() <= TOL["bf16"]
+    assert (whole[99:].double() - dec.double()).abs().max().item() <= TOL["bf16"]
+
+
+def test_prefill_reports_impossible_chunks():
+    ctxs = [20]
+    bt, kc, vc, q, qs = _build(ctxs, [20], 4, 4, 64, torch.float16, seed=9)
+    out = torch.empty(20, 4, 64, dtype=torch.float16, device="cuda")
+    # 20 new tokens but a context of only 10: impossible, reported, nothing faults.
+    pa.pa_prefill(out, q.cuda(), kc, vc, bt.cuda(), qs.cuda(), torch.tensor([10], dtype=torch.int32).cuda(), 20, 0.1, 4)
+    assert pa.pa_read_device_error(clear=True) & pa.PA_DEVERR_CTX_RANGE

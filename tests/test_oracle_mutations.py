@@ -126,3 +126,45 @@ def test_free_list_never_reusing_is_caught():
         a = fl.alloc()
         fl.free(a)
         assert fl.num_free == 3
+
+
+def test_prefill_without_causal_mask_is_caught():
+    from tests import test_oracle_prefill as TPF
+
+    def no_mask(q, k_pool, v_pool, bt, qs, lens, scale, hkv, kv_dtype, block_size=16):
+        q = np.asarray(q, dtype=np.float64)
+        out = np.zeros_like(q)
+        G = q.shape[1] // hkv
+        for s in range(len(lens)):
+            n = int(lens[s])
+            for hk in range(hkv):
+                K = attention.gather_context(k_pool, bt[s], n, hk, kv_dtype)
+                V = attention.gather_context(v_pool, bt[s], n, hk, kv_dtype)
+                for r in range(int(qs[s]), int(qs[s + 1])):
+                    for h in range(hk * G, (hk + 1) * G):
+                        out[r, h] = attention.attend(q[r, h], K, V, scale)  # every key, no diagonal
+        return out
+    with pytest.raises(AssertionError):
+        TPF.check_prefill_vs_sdpa(no_mask)
+
+
+def test_prefill_excluding_the_diagonal_is_caught():
+    from tests import test_oracle_prefill as TPF
+
+    def strict(q, k_pool, v_pool, bt, qs, lens, scale, hkv, kv_dtype, block_size=16):
+        q = np.asarray(q, dtype=np.float64)
+        out = np.zeros_like(q)
+        G = q.shape[1] // hkv
+        for s in range(len(lens)):
+            n = int(lens[s])
+            start = n - (int(qs[s + 1]) - int(qs[s]))
+            for hk in range(hkv):
+                K = attention.gather_context(k_pool, bt[s], n, hk, kv_dtype)
+                V = attention.gather_context(v_pool, bt[s], n, hk, kv_dtype)
+                for i, r in enumerate(range(int(qs[s]), int(qs[s + 1]))):
+                    p = max(start + i, 1)
+                    for h in range(hk * G, (hk + 1) * G):
+                        out[r, h] = attention.attend(q[r, h], K[:p], V[:p], scale)  # misses itself
+        return out
+    with pytest.raises(AssertionError):
+        TPF.check_prefill_vs_sdpa(strict)
