@@ -63,6 +63,25 @@ def dist_env():
     return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
 
 
+def max_over_ranks(value_ms: float, device=None) -> float:
+    """The slowest rank's time: every rank passes its own device time, all get the maximum.
+
+    Replicas run the same batch on every GPU with no exchange step, so the job's throughput is the
+    units all ranks processed over the slowest rank's time.
+    """
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return value_ms
+    t = torch.tensor([value_ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(bytes_per_rank_step: int, world: int, max_ms_per_step: float) -> float:
+    """Whole-job GB/s: all ranks' bytes per step over the slowest rank's step time."""
+    return bytes_per_rank_step * world / (max_ms_per_step / 1e3) / 1e9
+
+
 # ---------------------------------------------------------------------------------------------
 # Clock sampling during the timed region (NVML, every 20 ms).
 # ---------------------------------------------------------------------------------------------
@@ -353,11 +372,7 @@ def run_ours(args, rank, world, local_rank):
         dec_ms = [ev[k][1].elapsed_time(ev[k][2]) for k in range(K)]
         k1_ms = [ev[k][0].elapsed_time(ev[k][1]) for k in range(K)]
     dev_err = pa.pa_read_device_error(clear=True)
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([total_ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, device)
     ms_per_step = total_ms / K
 
     # ---- end to end through the C ABI with host buffers --------------------------------------
@@ -400,13 +415,8 @@ def run_ours(args, rank, world, local_rank):
         s1.record()
         torch.cuda.synchronize(device)
         barrier()
-        e_ms = s0.elapsed_time(s1)
-        if world > 1:
-            import torch.distributed as dist
-            t = torch.tensor([e_ms], device=device)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
-        e2e = {"value": round(kv_bytes * world / (e_ms / Ke / 1e3) / 1e9, 1), "unit": "GB/s",
+        e_ms = max_over_ranks(s0.elapsed_time(s1), device)
+        e2e = {"value": round(job_throughput(kv_bytes, world, e_ms / Ke), 1), "unit": "GB/s",
                "ms_per_step": round(e_ms / Ke, 5), "steps": Ke, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h,
                "note": "per step: one pinned H2D copy of the packed inputs (q, new K/V, slots, block tables, "
@@ -423,7 +433,7 @@ def run_ours(args, rank, world, local_rank):
     dec_avg_s = statistics.mean(dec_ms) / 1e3
     achieved = kv_bytes / dec_avg_s / 1e9
     traffic = ncu_traffic(args.workload)
-    value = kv_bytes * world / (ms_per_step / 1e3) / 1e9
+    value = job_throughput(kv_bytes, world, ms_per_step)
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline_sample(w)
