@@ -206,6 +206,8 @@ size_t pa_decode_cascade_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, 
  *   block_tables  [B, max_blocks] I32; query_start [B + 1] I32; context_lens [B] I32: tokens of
  *                 sequence s including the chunk (n_s <= context_lens[s] <= 16 * max_blocks).
  *   max_query_len host-known bound on n_s (sizes the grid without a device read).
+ *   kernel        -1 = choose (tcgen05 when D = 128 and Hq / Hkv divides 128), 0 = warp-level mma.sync
+ *                 tiles, 1 = tcgen05 (5th-generation tensor cores, accumulators in tensor memory).
  * Row i of sequence s is position p = context_lens[s] - n_s + i and sees positions 0 .. p:
  * out = softmax(scale * q K[0..p]^T) V[0..p], float32 accumulation, rounded to nearest even.
  * Violations only the device can see (n_s > context_lens[s], n_s > max_query_len) set
@@ -215,7 +217,7 @@ size_t pa_decode_cascade_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, 
  */
 int pa_prefill(pa_tensor* out, const pa_tensor* q, const pa_tensor* k_cache, const pa_tensor* v_cache,
                const pa_tensor* block_tables, const pa_tensor* query_start, const pa_tensor* context_lens,
-               int32_t max_query_len, float scale, int32_t num_kv_heads, void* stream);
+               int32_t max_query_len, float scale, int32_t num_kv_heads, int32_t kernel, void* stream);
 
 /* Partition size pa_decode uses when opts->partition_tokens == 0 and a workspace is given
  * (0 = no split: the batch's B * Hkv (sequence, KV head) units already fill the GPU and every

@@ -81,7 +81,7 @@ def _load() -> ctypes.CDLL:
         "pa_decode_cascade": (ctypes.c_int, [P, P, P, P, P, P, P, P, P, I32, F32, I32,
                                              ctypes.POINTER(PaDecodeOpts), VP]),
         "pa_decode_cascade_workspace_bytes": (SZ, [I32, I32, I32, I32, I32, I32, I32]),
-        "pa_prefill": (ctypes.c_int, [P, P, P, P, P, P, P, I32, F32, I32, VP]),
+        "pa_prefill": (ctypes.c_int, [P, P, P, P, P, P, P, I32, F32, I32, I32, VP]),
         "pa_decode_no_alloc": (ctypes.c_int, [P, P, P, P, P, P, F32, I32, ctypes.POINTER(PaDecodeOpts), VP]),
         "pa_decode_partition_tokens": (I32, [I32, I32, I32]),
         "pa_decode_workspace_bytes": (SZ, [I32, I32, I32, I32, I32, I32]),
@@ -255,13 +255,13 @@ def pa_decode_cascade_workspace_bytes(num_seqs: int, num_q_heads: int, num_kv_he
 
 def pa_prefill(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
                block_tables: torch.Tensor, query_start: torch.Tensor, context_lens: torch.Tensor, max_query_len: int,
-               scale: float, num_kv_heads: int, stream=None) -> None:
+               scale: float, num_kv_heads: int, kernel: int = -1, stream=None) -> None:
     """Causal attention of each sequence's new tokens over its paged context (see include/pa.h)."""
     args = [as_pa_tensor(out, "out"), as_pa_tensor(q, "q"), as_pa_tensor(k_cache, "k_cache"),
             as_pa_tensor(v_cache, "v_cache"), as_pa_tensor(block_tables, "block_tables"),
             as_pa_tensor(query_start, "query_start"), as_pa_tensor(context_lens, "context_lens")]
     _check(_lib.pa_prefill(*[ctypes.byref(a) for a in args], int(max_query_len), float(scale), int(num_kv_heads),
-                           ctypes.c_void_p(_stream_handle(stream))), "pa_prefill")
+                           int(kernel), ctypes.c_void_p(_stream_handle(stream))), "pa_prefill")
 
 
 # Size of the library's built-in scratch array used by pa_decode_no_alloc (PA_NO_ALLOC_SCRATCH_BYTES).

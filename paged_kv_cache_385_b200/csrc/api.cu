@@ -116,6 +116,23 @@ int encode_pool_map(CUtensorMap* map, const pa_tensor* cache, int esz) {
   return PA_OK;
 }
 
+// q [T, Hq, D] (16-bit) as a 3-D tensor {D, Hq, T}, boxes of 64 x G x (128 / G): 128 rows of 128
+// bytes (tokens x group heads of one KV head), 128-byte swizzle.
+int encode_q_map(CUtensorMap* map, const pa_tensor* q, int group) {
+  auto fn = encode_fn();
+  if (!fn) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(q->shape[2]), static_cast<cuuint64_t>(q->shape[1]),
+                              static_cast<cuuint64_t>(q->shape[0])};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(q->stride[1] * 2), static_cast<cuuint64_t>(q->stride[0] * 2)};
+  const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(group), static_cast<cuuint32_t>(128 / group)};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, q->dtype == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
+                  q->data, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled (q) failed (%d)", static_cast<int>(r));
+  return PA_OK;
+}
+
 uint32_t* library_error_word() {
   static uint32_t* words[64] = {nullptr};
   int dev = 0;
@@ -572,7 +589,7 @@ size_t pa_decode_cascade_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, 
 
 int pa_prefill(pa_tensor* out, const pa_tensor* q, const pa_tensor* k_cache, const pa_tensor* v_cache,
                const pa_tensor* block_tables, const pa_tensor* query_start, const pa_tensor* context_lens,
-               int32_t max_query_len, float scale, int32_t num_kv_heads, void* stream) {
+               int32_t max_query_len, float scale, int32_t num_kv_heads, int32_t kernel, void* stream) {
   int st;
   if ((st = check_tensor(out, "out", 3)) || (st = check_tensor(q, "q", 3)) || (st = check_tensor(k_cache, "k_cache", 4)) ||
       (st = check_tensor(v_cache, "v_cache", 4)) || (st = check_tensor(block_tables, "block_tables", 2)) ||
@@ -634,7 +651,18 @@ int pa_prefill(pa_tensor* out, const pa_tensor* q, const pa_tensor* k_cache, con
   CUtensorMap km, vm;
   if ((st = encode_pool_map(&km, k_cache, 2)) || (st = encode_pool_map(&vm, v_cache, 2))) return st;
   const pa::KvType kv = cd == PA_BF16 ? pa::KvType::BF16 : pa::KvType::F16;
-  cudaError_t e = pa::launch_prefill(kv, static_cast<int>(D), km, vm, p, max_query_len, static_cast<cudaStream_t>(stream));
+  const int G = static_cast<int>(Hq / num_kv_heads);
+  if (kernel < -1 || kernel > 1) return fail(PA_ERR_INVALID_ARG, "kernel must be -1, 0 or 1");
+  const bool tc_ok = pa::prefill_tc_supported(static_cast<int>(D), G);
+  if (kernel == 1 && !tc_ok) return fail(PA_ERR_UNSUPPORTED, "the tcgen05 prefill needs head_dim 128 and a group dividing 128");
+  cudaError_t e;
+  if (kernel == 1 || (kernel == -1 && tc_ok)) {
+    CUtensorMap qm;
+    if ((st = encode_q_map(&qm, q, G))) return st;
+    e = pa::launch_prefill_tc(kv, qm, km, vm, p, max_query_len, static_cast<cudaStream_t>(stream));
+  } else {
+    e = pa::launch_prefill(kv, static_cast<int>(D), km, vm, p, max_query_len, static_cast<cudaStream_t>(stream));
+  }
   if (e != cudaSuccess) return fail(PA_ERR_CUDA, "prefill launch: %s", cudaGetErrorString(e));
   return ok();
 }

@@ -116,6 +116,10 @@ cudaError_t launch_prefix(KvType kv, int head_dim, const CUtensorMap& k_map, con
                           const MqParams& p, cudaStream_t stream);
 cudaError_t launch_prefill(KvType kv, int head_dim, const CUtensorMap& k_map, const CUtensorMap& v_map,
                            const MqParams& p, int max_query_len, cudaStream_t stream);
+// tcgen05 prefill (prefill_tc.cu): q_map is a 3-D map over q [T, Hq, D] with box {64, G, 128 / G}.
+bool prefill_tc_supported(int head_dim, int group);
+cudaError_t launch_prefill_tc(KvType kv, const CUtensorMap& q_map, const CUtensorMap& k_map, const CUtensorMap& v_map,
+                              const MqParams& p, int max_query_len, cudaStream_t stream);
 
 struct CopyParams {
   void* k_cache;

@@ -40,21 +40,43 @@ def _oracle(bt, kc, vc, q, qs, ctxs, scale, hkv, kvd):
     return attention.prefill_paged(q.double().numpy(), kb, vb, bt.numpy(), qs.tolist(), ctxs, scale, hkv, kvd)
 
 
-@pytest.mark.parametrize("ctxs,news,hq,hkv,d,dtype", [
+CASES = [
     ([37, 160, 90], [37, 16, 70], 8, 2, 128, torch.bfloat16),
     ([1, 64, 200, 33], [1, 64, 5, 33], 4, 4, 64, torch.float16),
     ([300, 129], [150, 129], 16, 2, 128, torch.float16),
-])
-def test_prefill_matches_oracle(ctxs, news, hq, hkv, d, dtype):
+    ([700, 5, 260], [400, 5, 131], 32, 8, 128, torch.bfloat16),
+    ([129, 40], [129, 40], 4, 4, 128, torch.float16),
+]
+
+
+@pytest.mark.parametrize("kernel", [0, 1])
+@pytest.mark.parametrize("ctxs,news,hq,hkv,d,dtype", CASES)
+def test_prefill_matches_oracle(ctxs, news, hq, hkv, d, dtype, kernel):
+    if kernel == 1 and d != 128:
+        pytest.skip("the tcgen05 prefill takes head_dim 128")
     bt, kc, vc, q, qs = _build(ctxs, news, hq, hkv, d, dtype, seed=sum(ctxs))
     out = torch.full((q.shape[0], hq, d), float("nan"), dtype=dtype, device="cuda")
     pa.pa_prefill(out, q.cuda(), kc, vc, bt.cuda(), qs.cuda(), torch.tensor(ctxs, dtype=torch.int32).cuda(),
-                  max(news), 1.0 / np.sqrt(d), hkv)
+                  max(news), 1.0 / np.sqrt(d), hkv, kernel=kernel)
     torch.cuda.synchronize()
     assert pa.pa_read_device_error(clear=True) == 0
     want = _oracle(bt, kc, vc, q, qs, ctxs, 1.0 / np.sqrt(d), hkv, "bf16" if dtype == torch.bfloat16 else "f16")
     err = float(np.max(np.abs(out.double().cpu().numpy() - want)))
     assert err <= TOL["bf16" if dtype == torch.bfloat16 else "f16"], err
+
+
+def test_tcgen05_and_warp_mma_prefill_agree():
+    ctxs, news, hq, hkv, d = [1000, 77], [1000, 77], 32, 8, 128
+    bt, kc, vc, q, qs = _build(ctxs, news, hq, hkv, d, torch.bfloat16, seed=31)
+    outs = []
+    for kernel in (0, 1):
+        out = torch.empty(q.shape[0], hq, d, dtype=torch.bfloat16, device="cuda")
+        pa.pa_prefill(out, q.cuda(), kc, vc, bt.cuda(), qs.cuda(), torch.tensor(ctxs, dtype=torch.int32).cuda(),
+                      max(news), d ** -0.5, hkv, kernel=kernel)
+        outs.append(out)
+    torch.cuda.synchronize()
+    assert pa.pa_read_device_error(clear=True) == 0
+    assert (outs[0].double() - outs[1].double()).abs().max().item() <= TOL["bf16"]
 
 
 def test_chunked_equals_whole_and_last_row_equals_decode():
