@@ -54,6 +54,8 @@ def parse():
     ap.add_argument("--op", choices=["step", "copy_blocks", "kv_utilization", "prefill"], default="step",
                     help="step: the decode step (the headline); copy_blocks: copy-on-write block copies; "
                          "kv_utilization: KV memory utilisation of the block allocator (host only)")
+    ap.add_argument("--prefix-kernel", type=int, default=-1,
+                    help="--step cascade: shared-prefix kernel, -1 library choice, 0 warp-level mma, 1 tcgen05")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args()
@@ -205,6 +207,7 @@ class Setup:
         self.partition_tokens_used = eff_pt if self.split else 0
         self.fused_step = True
         self.cascade_step = False
+        self.prefix_kernel = -1
         self.launches_per_step = 2 + (1 if self.split else 0)
         torch.cuda.synchronize(device)
 
@@ -224,7 +227,7 @@ class Setup:
                                                           self.max_ctx, w.shared_prefix_tokens, 0)
             self._casc_ws = torch.empty(n, dtype=torch.uint8, device=self.device)
             self._casc_opts = self.pa.decode_opts(max_context_len=self.max_ctx, workspace=self._casc_ws,
-                                                  kernel=self.kernel)
+                                                  kernel=self.kernel, prefix_kernel=self.prefix_kernel)
         self.pa.pa_decode_cascade(self.out, self.q, self.new_k, self.new_v, self.new_slots, self.k_cache,
                                   self.v_cache, self.bt, self.lens, w.shared_prefix_tokens, w.scale, w.num_kv_heads,
                                   opts=self._casc_opts, stream=stream)
@@ -326,7 +329,14 @@ def run_ours(args, rank, world, local_rank):
     st.cascade_step = args.step == "cascade"
     if st.cascade_step and not w.shared_prefix_tokens:
         raise SystemExit("--step cascade needs a workload with a shared prefix (prefix_gqa)")
-    st.launches_per_step = 3 if st.cascade_step else (1 if st.fused_step else 2) + (1 if st.split else 0)
+    st.prefix_kernel = args.prefix_kernel
+    if st.cascade_step:
+        # prefix kernel + suffix decode (+ the partition merge when the suffix itself splits)
+        span = max(st.max_ctx - w.shared_prefix_tokens, 1)
+        spt = st.pa.pa_decode_partition_tokens(w.num_seqs, w.num_kv_heads, span)
+        st.launches_per_step = 2 + (1 if spt > 0 and -(-span // spt) > 1 else 0)
+    else:
+        st.launches_per_step = (1 if st.fused_step else 2) + (1 if st.split else 0)
     kv_bytes = W.kv_bytes_read(w, st.lens_host)
     K, Wm = args.steps, max(3, args.warmup)
 
@@ -462,6 +472,8 @@ def run_ours(args, rank, world, local_rank):
                    "context_lens": "fixed 2048" if w.name == "llama7b_mha" else str(w.ctx),
                    "pool_blocks": w.num_blocks, "kv_bytes_per_step": kv_bytes,
                    "partition_tokens": st.partition_tokens_used, "kernel": "tensor-core" if args.kernel != 0 else "cuda-core",
+                   **({"prefix_kernel": "warp-level mma" if args.prefix_kernel == 0 else "tcgen05"}
+                      if st.cascade_step else {}),
                    "l2": f"inputs larger than L2: {kv_bytes / 1e9:.2f} GB of KV per step vs 126 MB L2, no flush",
                    "parallelism": f"replicas x{world}"},
         "roofline": {"bound": "hbm", "kernel": ("pa_decode_cascade (prefix + suffix decode + merge kernels)"
@@ -536,8 +548,10 @@ def run_prefill(args, rank, world, local_rank):
     flops = B * Hq * 2 * 2 * D * (n * (n + 1) // 2)
     K, Wm = max(5, args.steps // 100), max(3, args.warmup)
 
+    kernel = 1 if args.kernel == -1 else args.kernel  # -1: the library's choice (tcgen05 here)
+
     def call():
-        pa.pa_prefill(out, q, kc, vc, btd, qs, lens, n, D ** -0.5, Hkv)
+        pa.pa_prefill(out, q, kc, vc, btd, qs, lens, n, D ** -0.5, Hkv, kernel=kernel)
 
     for _ in range(Wm):
         call()
@@ -566,7 +580,7 @@ def run_prefill(args, rank, world, local_rank):
                        "flops_per_call": flops},
             "roofline": {"bound": "tensor", "achieved": round(tflops, 1), "peak": peak, "unit": "TFLOP/s",
                          "frac": round(tflops / peak, 4), "traffic": None, "peak_source": src,
-                         "note": "warp-level mma.sync m16n8k16; the peak is a tcgen05 cuBLAS figure"},
+                         "kernel": "tcgen05 (tensor memory accumulators)" if kernel == 1 else "warp-level mma.sync"},
             "gpu_launches": K, "clocks": clocks.summary()}), flush=True)
 
 

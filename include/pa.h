@@ -95,6 +95,10 @@ typedef struct pa_decode_opts {
   size_t workspace_bytes;
   int32_t kernel;           /* -1 = choose; 0 = CUDA-core FMA kernel; 1 = tensor-core (mma) kernel     */
   int32_t* error_word;      /* device int32 that receives PA_DEVERR_* bits; NULL = library's own word  */
+  int32_t prefix_kernel;    /* pa_decode_cascade's shared-prefix kernel: -1 = choose (tcgen05 when
+                               head_dim is 128, the group divides 128 and q rows are 16-B aligned);
+                               0 = warp-level mma kernel; 1 = tcgen05 kernel (PA_ERR_UNSUPPORTED
+                               when those conditions fail)                                             */
 } pa_decode_opts;
 
 /* Fill opts with the defaults (scales 1, everything else automatic). */

@@ -57,7 +57,7 @@ class PaDecodeOpts(ctypes.Structure):
     _fields_ = [("k_scale", ctypes.c_float), ("v_scale", ctypes.c_float), ("max_context_len", ctypes.c_int32),
                 ("partition_tokens", ctypes.c_int32), ("workspace", ctypes.c_void_p),
                 ("workspace_bytes", ctypes.c_size_t), ("kernel", ctypes.c_int32),
-                ("error_word", ctypes.c_void_p)]
+                ("error_word", ctypes.c_void_p), ("prefix_kernel", ctypes.c_int32)]
 
 
 class PagedAttentionError(RuntimeError):
@@ -176,7 +176,7 @@ def pa_copy_blocks(k_cache: torch.Tensor, v_cache: torch.Tensor, block_mapping: 
 
 def decode_opts(k_scale: float = 1.0, v_scale: float = 1.0, max_context_len: int = 0, partition_tokens: int = 0,
                 workspace: Optional[torch.Tensor] = None, kernel: int = -1,
-                error_word: Optional[torch.Tensor] = None) -> PaDecodeOpts:
+                error_word: Optional[torch.Tensor] = None, prefix_kernel: int = -1) -> PaDecodeOpts:
     o = PaDecodeOpts()
     _lib.pa_decode_opts_init(ctypes.byref(o))
     o.k_scale = k_scale
@@ -189,6 +189,7 @@ def decode_opts(k_scale: float = 1.0, v_scale: float = 1.0, max_context_len: int
         o.workspace = workspace.data_ptr()
         o.workspace_bytes = workspace.numel() * workspace.element_size()
     o.kernel = int(kernel)
+    o.prefix_kernel = int(prefix_kernel)
     if error_word is not None:
         if not error_word.is_cuda or error_word.dtype != torch.int32:
             raise ValueError("error_word must be a CUDA int32 tensor")

@@ -204,6 +204,7 @@ void pa_decode_opts_init(pa_decode_opts* o) {
   o->k_scale = 1.0f;
   o->v_scale = 1.0f;
   o->kernel = -1;
+  o->prefix_kernel = -1;
 }
 
 int32_t pa_decode_partition_tokens(int32_t num_seqs, int32_t num_kv_heads, int32_t max_context_len) {
@@ -390,12 +391,20 @@ static int decode_impl(pa_tensor* out, const pa_tensor* q, const pa_tensor* k_ca
   // Cascade: the shared prefix goes to the prefix kernel (n_pre chunks); this grid covers the suffix.
   const bool cascade = prefix_tokens > 0;
   int64_t n_pre = 0;
+  bool use_tc_prefix = false;
   if (cascade) {
     if (cd == PA_E4M3) return fail(PA_ERR_UNSUPPORTED, "shared-prefix decode takes F16 or BF16 caches");
     if (prefix_tokens % 16) return fail(PA_ERR_INVALID_ARG, "shared_prefix_tokens must be a multiple of 16");
     if (prefix_tokens > max_blocks * 16)
       return fail(PA_ERR_INVALID_ARG, "shared_prefix_tokens %d exceeds the block-table width", prefix_tokens);
     n_pre = (prefix_tokens + pa::kPrefixChunkTokens - 1) / pa::kPrefixChunkTokens;
+    if (opts.prefix_kernel < -1 || opts.prefix_kernel > 1)
+      return fail(PA_ERR_INVALID_ARG, "opts.prefix_kernel must be -1, 0 or 1");
+    const bool tc_ok = pa::prefill_tc_supported(static_cast<int>(D), static_cast<int>(G)) && q->stride[2] == 1 &&
+                       q->stride[1] % 8 == 0 && q->stride[0] % 8 == 0 && aligned(q->data, 16);
+    if (opts.prefix_kernel == 1 && !tc_ok)
+      return fail(PA_ERR_UNSUPPORTED, "the tcgen05 prefix kernel needs head_dim 128, a group dividing 128 and 16-byte aligned q rows");
+    use_tc_prefix = opts.prefix_kernel == 1 || (opts.prefix_kernel == -1 && tc_ok);
   }
   const int64_t span_max = std::max<int64_t>(max_ctx - (cascade ? prefix_tokens : 0), 0);
   if (pt == 0) {
@@ -432,6 +441,7 @@ static int decode_impl(pa_tensor* out, const pa_tensor* q, const pa_tensor* k_ca
   p.ws_parts = static_cast<int32_t>(ws_parts);
   p.always_partials = cascade ? 1 : 0;
   p.merge_prefix_inline = cascade && P == 1 ? 1 : 0;
+  p.late_dependency_wait = cascade ? 1 : 0;
   p.err = opts.error_word ? reinterpret_cast<uint32_t*>(opts.error_word) : library_error_word();
   if (!p.err) return fail(PA_ERR_CUDA, "no device error word (no current CUDA device?)");
   if (ws_parts > 1) {
@@ -508,7 +518,13 @@ static int decode_impl(pa_tensor* out, const pa_tensor* q, const pa_tensor* k_ca
     pp.ws_ml = p.ws_ml;
     pp.ws_parts = p.ws_parts;
     pp.err = p.err;
-    e = pa::launch_prefix(cfg.kv, cfg.head_dim, km, vm, pp, s);
+    if (use_tc_prefix) {
+      CUtensorMap qm;
+      if ((st = encode_q_map(&qm, q, static_cast<int>(G)))) return st;
+      e = pa::launch_prefix_tc(cfg.kv, qm, km, vm, pp, s);
+    } else {
+      e = pa::launch_prefix(cfg.kv, cfg.head_dim, km, vm, pp, s);
+    }
     if (e != cudaSuccess) return fail(PA_ERR_CUDA, "prefix launch: %s", cudaGetErrorString(e));
   }
   e = pa::launch_decode(cfg, km, vm, p, s);

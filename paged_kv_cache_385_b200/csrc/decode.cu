@@ -471,9 +471,11 @@ __global__ void __launch_bounds__(Cfg<KV, QT, D, NT, KIND, OCC>::kThreads, Cfg<K
   const int part = blockIdx.x, hk = blockIdx.y, s = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // Launched as a programmatic dependent: everything this grid reads may come from the previous
-  // kernel on the stream, so wait for it first. The next kernel (partition merge, next step) is let
-  // in once every CTA has finished its page loop (below), when SM slots start to free up.
-  pdl_wait();
+  // kernel on the stream, so wait for it first (cascade: only before the prefix partials are read).
+  // The next kernel (partition merge, next step) is let in once every CTA has finished its page loop
+  // (below), when SM slots start to free up.
+  const bool late_wait = p.late_dependency_wait != 0;
+  if (!late_wait) pdl_wait();
   const int G = p.group;
   const int Hq = p.num_kv_heads * G;
   const int PT = p.partition_tokens;
@@ -489,7 +491,10 @@ __global__ void __launch_bounds__(Cfg<KV, QT, D, NT, KIND, OCC>::kThreads, Cfg<K
   }
   const int ctx_eff = start + span;  // tokens [0, ctx_eff) exist for this grid's bookkeeping
   const int nparts = (span + PT - 1) / PT;
-  if (part >= max(nparts, 1)) return;
+  if (part >= max(nparts, 1)) {
+    if (late_wait) pdl_wait();
+    return;
+  }
 
   // pa_decode_step: the CTA holding the sequence's last partition writes head hk's new K/V row
   // (position ctx - 1) into its slot before any of its page copies start. No other CTA reads that
@@ -531,6 +536,7 @@ __global__ void __launch_bounds__(Cfg<KV, QT, D, NT, KIND, OCC>::kThreads, Cfg<K
   }
 
   typedef uint16_t out_t;
+  if (span == 0 && late_wait) pdl_wait();
   if (span == 0 && p.merge_prefix_inline) {
     // Nothing past the shared prefix: the output is the merge of the prefix partials alone.
     for (int idx = threadIdx.x; idx < G * D; idx += C::kThreads) {
@@ -676,6 +682,7 @@ __global__ void __launch_bounds__(Cfg<KV, QT, D, NT, KIND, OCC>::kThreads, Cfg<K
   }
   const int any_fail = __syncthreads_or(!ok);
   pdl_launch_dependents();
+  if (late_wait) pdl_wait();  // the prefix partials (and the prefix grid's completion) from here on
 
   // ---- merge the warps in fixed order -----------------------------------------------------
   if constexpr (KIND == 1) {

@@ -41,6 +41,11 @@ struct DecodeParams {
   // Cascade with an unsplit suffix: the decode CTA merges the prefix partials (slots [0, part_offset))
   // with its own result and writes the output; no merge kernel runs.
   int32_t merge_prefix_inline;
+  // Cascade: the kernel before this grid on the stream is the prefix kernel, which lets it launch
+  // only after its own wait on the kernel before that, so pages, q and tables are already final when
+  // this grid starts. It therefore waits for the prefix grid (griddepcontrol.wait) only before it
+  // reads the prefix partials and before every exit, and its page loop overlaps the prefix kernel.
+  int32_t late_dependency_wait;
   // Fused new-token write (pa_decode_step); new_k == nullptr for plain pa_decode.
   const void* new_k;         // [B, Hkv, D] f16/bf16
   const void* new_v;
@@ -120,6 +125,9 @@ cudaError_t launch_prefill(KvType kv, int head_dim, const CUtensorMap& k_map, co
 bool prefill_tc_supported(int head_dim, int group);
 cudaError_t launch_prefill_tc(KvType kv, const CUtensorMap& q_map, const CUtensorMap& k_map, const CUtensorMap& v_map,
                               const MqParams& p, int max_query_len, cudaStream_t stream);
+// The same kernel in shared-prefix mode: q_map over q [B, Hq, D], partials to ws slots 0 .. num_chunks-1.
+cudaError_t launch_prefix_tc(KvType kv, const CUtensorMap& q_map, const CUtensorMap& k_map, const CUtensorMap& v_map,
+                             const MqParams& p, cudaStream_t stream);
 
 struct CopyParams {
   void* k_cache;

@@ -61,6 +61,9 @@ __global__ void __launch_bounds__(PCfg<KV, D>::kThreads) mq_kernel(const __grid_
   const int G = p.group;
   const int Hq = p.num_kv_heads * G;
   pdl_wait();
+  // Shared-prefix mode: the suffix decode after this grid waits for it only at its merge, so it may
+  // launch now and overlap its page loop with this kernel.
+  if constexpr (!kPrefill) pdl_launch_dependents();
 
   // Rows and pages of this CTA.
   int chunk = 0, s_seq = 0, num_rows, j0, npages, q_row0 = 0, start = 0;
@@ -289,7 +292,7 @@ __global__ void __launch_bounds__(PCfg<KV, D>::kThreads) mq_kernel(const __grid_
     __syncwarp();
     if (lane == 0) mbar_arrive(empty0 + 8 * st);
   }
-  pdl_launch_dependents();
+  if constexpr (kPrefill) pdl_launch_dependents();
   if (!ok) return;
 
   l_lo += __shfl_xor_sync(kFull, l_lo, 1);

@@ -1,12 +1,16 @@
-// Chunked prefill over paged KV with 5th-generation tensor cores (tcgen05 + tensor memory).
+// Multi-query attention over paged KV with 5th-generation tensor cores (tcgen05 + tensor memory),
+// in two modes:
+// * Chunked prefill (pa_prefill; notes page, kernels section: FlashAttention adapted to paged KV;
+//   "vLLM 前世今生" §5.4 chunked prefill): row (new token i, group head g) of sequence s is position
+//   p = start + i and attends over positions 0 .. p of its KV head.
+// * Shared prefix (pa_decode_cascade; "vLLM 前世今生" §3.2, several sequences mapping the same
+//   physical blocks): row (sequence s, group head g) holds that sequence's decode query; a CTA takes
+//   one chunk of the prefix pages every block table shares and writes the rows' partial softmax
+//   state (m, l, unnormalised acc) to the split workspace, merged later with the sequence's suffix.
 //
-// What is computed: as pa_prefill (notes page, kernels section: FlashAttention adapted to paged KV;
-// "vLLM 前世今生" §5.4 chunked prefill): row (new token i, group head g) of sequence s is position
-// p = start + i and attends over positions 0 .. p of its KV head.
-//
-// CTA = 128 query rows (tokens x group heads of one sequence and KV head). Per block of 128 keys
-// (8 pages), with the block's K and V staged by TMA in 128-byte-swizzled shared memory:
-//   S[128 x 128] = Q . K^T      tcgen05.mma kind::f16, A = Q (K-major), B = K (K-major), D in TMEM
+// CTA = 128 query rows of one KV head. Per block of KEYS keys (KEYS / 16 pages), with the block's K
+// and V staged by TMA in 128-byte-swizzled shared memory:
+//   S[128 x KEYS] = Q . K^T     tcgen05.mma kind::f16, A = Q (K-major), B = K (K-major), D in TMEM
 //   softmax                     4 warps, one row per thread, S read from TMEM (tcgen05.ld), running
 //                               max / sum in registers, P written (bf16/f16) to shared memory, O
 //                               rescaled in TMEM when a row's max moved
@@ -17,52 +21,93 @@
 #include "pa_device.cuh"
 #include "tc05.cuh"
 
+#ifndef PA_PREFILL_TC_KEYS
+#define PA_PREFILL_TC_KEYS 64
+#endif
+
 namespace pa {
 namespace {
 
 constexpr int kD = 128;
 constexpr int kRows = 128;   // query rows per CTA
-constexpr int kKeys = 128;   // keys per block
 constexpr int kThreads = 192;
 constexpr uint32_t kHalf = 16384;  // one 64-element (128-byte) column half of a 128-row tile
 constexpr uint32_t kTile = 2 * kHalf;
-constexpr uint32_t kQOff = 0;
-constexpr uint32_t kStageOff = kTile;                 // stage s: K at kStageOff + s*2*kTile, V after it
-constexpr uint32_t kPOff = kStageOff + 4 * kTile;     // P tile
-constexpr uint32_t kBarOff = kPOff + kTile;           // mbarriers
-constexpr uint32_t kSmemBytes = 1024 + kBarOff + 128;
-// barrier slots (8 bytes each)
-enum { kQFull = 0, kKvFull0 = 1, kKvEmpty0 = 3, kSFull = 5, kPFull = 6, kODone = 7, kAllDone = 8, kTmemSlot = 9 };
 
-template <bool kBf16>
-__global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap,
-                                                                  const __grid_constant__ CUtensorMap kmap,
-                                                                  const __grid_constant__ CUtensorMap vmap,
-                                                                  const MqParams p) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+// KEYS keys per block: 128 (one CTA per SM, 2 stages of 64 KB) or 64 (two CTAs per SM sharing the
+// tensor core, so one CTA's softmax overlaps the other's MMAs: 112 KB of shared memory each).
+template <int KEYS>
+struct TcCfg {
+  static constexpr uint32_t kHalfKV = KEYS * 128;            // a 64-element column half of a K or V tile
+  static constexpr uint32_t kTileKV = 2 * kHalfKV;
+  static constexpr uint32_t kQOff = 0;
+  static constexpr uint32_t kStageOff = kTile;                // stage s: K at + s * 2 * kTileKV, V after it
+  static constexpr uint32_t kPOff = kStageOff + 4 * kTileKV;  // P tile: KEYS / 64 halves of 128 x 128 B
+  static constexpr uint32_t kBarOff = kPOff + (KEYS / 64) * kHalf;
+  static constexpr uint32_t kSmemBytes = kBarOff + 128;
+  static constexpr int kMinBlocks = KEYS == 64 ? 2 : 1;
+};
+// barrier slots (8 bytes each)
+enum { kQFull = 0, kKvFull0 = 1, kKvEmpty0 = 3, kSFull0 = 5, kPFull = 7, kODone = 8, kAllDone = 9, kTmemSlot = 10 };
+// O is rescaled only when a row's running max grows by more than this (log2 units); until then P and
+// the row sum keep the older reference, so the result is unchanged and P stays below 2^8.
+constexpr float kLazyRescale = 8.f;
+
+template <bool kBf16, int KEYS, bool kPrefix>
+__global__ void __launch_bounds__(kThreads, TcCfg<KEYS>::kMinBlocks)
+    prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
+                      const __grid_constant__ CUtensorMap vmap, const MqParams p) {
+  using C = TcCfg<KEYS>;
+  constexpr int kKeys = KEYS;
+  constexpr uint32_t kHalfKV = C::kHalfKV, kTileKV = C::kTileKV, kQOff = C::kQOff, kStageOff = C::kStageOff;
+  constexpr uint32_t kPOff = C::kPOff, kBarOff = C::kBarOff;
+  extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t base = smem_u32(smem);
+  if (base & 1023u) {  // the swizzled tiles need 1024-byte alignment; never seen, but do not guess
+    if (threadIdx.x == 0) atomicOr(p.err, 4u);
+    return;
+  }
   const uint32_t bar = base + kBarOff;
   auto B = [&](int i) { return bar + 8u * i; };
 
+  // Prefill: blockIdx.z is the sequence. Prefix: blockIdx.z is the prefix chunk and row R of the
+  // grid is (sequence R / G, group head R % G).
   const int tile = blockIdx.x, hk = blockIdx.y, s = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = p.group;
   pdl_wait();
+  // Prefix mode: the suffix decode after this grid reads nothing of it until its merge (where it
+  // waits for this grid), so let it launch now and overlap its page loop with these MMAs.
+  if constexpr (kPrefix) pdl_launch_dependents();
 
-  const int q_row0 = p.query_start[s];
-  const int n_new = p.query_start[s + 1] - q_row0;
-  const int num_rows = n_new * G;
-  if (tile * kRows >= num_rows) return;
-  const int ctx = p.context_lens[s];
-  const int start = ctx - n_new;
-  if (start < 0 || ctx > p.max_blocks * 16) {
-    if (threadIdx.x == 0) atomicOr(p.err, 8u);
-    return;
+  int q_row0, num_rows, start, key0, max_lim;  // keys [key0, key0 + max_lim) of the KV head
+  const int32_t* bt;
+  if constexpr (kPrefix) {
+    q_row0 = 0;
+    num_rows = p.num_seqs * G;
+    if (tile * kRows >= num_rows) return;
+    start = 0;
+    key0 = s * p.chunk_tokens;
+    max_lim = min(p.chunk_tokens, p.prefix_tokens - key0);
+    if (max_lim <= 0) return;
+    bt = p.block_tables + key0 / 16;  // sequence 0's row; every sequence must map the same blocks
+  } else {
+    q_row0 = p.query_start[s];
+    const int n_new = p.query_start[s + 1] - q_row0;
+    num_rows = n_new * G;
+    if (tile * kRows >= num_rows) return;
+    const int ctx = p.context_lens[s];
+    start = ctx - n_new;
+    if (start < 0 || ctx > p.max_blocks * 16) {
+      if (threadIdx.x == 0) atomicOr(p.err, 8u);
+      return;
+    }
+    if (tile == 0 && threadIdx.x == 0 && num_rows > static_cast<int>(gridDim.x) * kRows) atomicOr(p.err, 8u);
+    const int last_row = min((tile + 1) * kRows, num_rows) - 1;
+    key0 = 0;
+    max_lim = start + last_row / G + 1;  // keys visible to the tile's last row
+    bt = p.block_tables + static_cast<int64_t>(s) * p.bt_stride;
   }
-  if (tile == 0 && threadIdx.x == 0 && num_rows > static_cast<int>(gridDim.x) * kRows) atomicOr(p.err, 8u);
-  const int last_row = min((tile + 1) * kRows, num_rows) - 1;
-  const int max_lim = start + last_row / G + 1;  // keys visible to the tile's last row
   const int npages = (max_lim + 15) / 16;
   const int nkb = (max_lim + kKeys - 1) / kKeys;
 
@@ -72,18 +117,22 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
     mbar_init(B(kKvFull0 + 1), 1);
     mbar_init(B(kKvEmpty0), 1);
     mbar_init(B(kKvEmpty0 + 1), 1);
-    mbar_init(B(kSFull), 1);
+    mbar_init(B(kSFull0), 1);
+    mbar_init(B(kSFull0 + 1), 1);
     mbar_init(B(kPFull), 4);
     mbar_init(B(kODone), 1);
     mbar_init(B(kAllDone), 1);
     fence_barrier_init();
   }
-  if (warp == 5) tc05::alloc(B(kTmemSlot), 256);
+  // TMEM: two S buffers of kKeys columns (QK of the next block runs while this one's softmax does),
+  // then O's 128 columns.
+  constexpr uint32_t kTmemCols = 2 * kKeys + kD <= 256 ? 256 : 512;
+  if (warp == 5) tc05::alloc(B(kTmemSlot), kTmemCols);
   tc05::fence_before_sync();
   __syncthreads();
   tc05::fence_after_sync();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + kBarOff + 8 * kTmemSlot);
-  const uint32_t tS = tmem, tO = tmem + 128;
+  const uint32_t tS0 = tmem, tO = tmem + 2 * kKeys;
   const uint64_t deadline = globaltimer_ns() + 2000000000ull;
   bool ok = true;
 
@@ -95,7 +144,6 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
       const int tok0 = q_row0 + tile * (kRows / G);
       tc05::tma_load_3d(base + kQOff, &qmap, B(kQFull), 0, hk * G, tok0);
       tc05::tma_load_3d(base + kQOff + kHalf, &qmap, B(kQFull), 64, hk * G, tok0);
-      const int32_t* bt = p.block_tables + static_cast<int64_t>(s) * p.bt_stride;
       const int oob_row = p.num_blocks * p.num_kv_heads * 16;  // a box starting here is all zero fill
       for (int j = 0; j < nkb && ok; ++j) {
         const int st = j & 1;
@@ -104,7 +152,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
           atomicOr(p.err, 4u);
           break;
         }
-        const uint32_t kdst = base + kStageOff + st * 2 * kTile, vdst = kdst + kTile;
+        const uint32_t kdst = base + kStageOff + st * 2 * kTileKV, vdst = kdst + kTileKV;
         // The block's 8 page ids are loaded together, then its 32 tile copies issued.
         int ys[kKeys / 16];
 #pragma unroll
@@ -122,13 +170,13 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             else atomicOr(p.err, 1u);
           }
         }
-        mbar_arrive_expect_tx(B(kKvFull0 + st), 2 * kTile);
+        mbar_arrive_expect_tx(B(kKvFull0 + st), 2 * kTileKV);
 #pragma unroll
         for (int i = 0; i < kKeys / 16; ++i) {
           const int y = ys[i];
           for (int u = 0; u < 2; ++u) {
-            tma_load_2d(kdst + u * kHalf + i * 2048, &kmap, B(kKvFull0 + st), u * 64, y);
-            tma_load_2d(vdst + u * kHalf + i * 2048, &vmap, B(kKvFull0 + st), u * 64, y);
+            tma_load_2d(kdst + u * kHalfKV + i * 2048, &kmap, B(kKvFull0 + st), u * 64, y);
+            tma_load_2d(vdst + u * kHalfKV + i * 2048, &vmap, B(kKvFull0 + st), u * 64, y);
           }
         }
       }
@@ -138,37 +186,42 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
     if (lane == 0) {
       constexpr uint32_t idesc_qk = tc05::idesc_f16(kBf16, kRows, kKeys, false, false);
       constexpr uint32_t idesc_pv = tc05::idesc_f16(kBf16, kRows, kD, false, true);
-      if (!mbar_wait_bounded(B(kQFull), 0, deadline)) ok = false;
-      for (int j = 0; j < nkb && ok; ++j) {
+      // S(j) = Q K(j)^T into S buffer j & 1.
+      auto issue_qk = [&](int j) -> bool {
         const int st = j & 1;
-        if (!mbar_wait_bounded(B(kKvFull0 + st), (j >> 1) & 1, deadline)) {
+        if (!mbar_wait_bounded(B(kKvFull0 + st), (j >> 1) & 1, deadline)) return false;
+        tc05::fence_after_sync();
+        const uint32_t kbase = base + kStageOff + st * 2 * kTileKV;
+#pragma unroll
+        for (int ks = 0; ks < kD / 16; ++ks) {  // 8 k-steps of 16 along d, 32 bytes apart in a half
+          const uint32_t cb = (ks & 3) * 32;
+          tc05::mma_f16(tS0 + st * kKeys, tc05::smem_desc_sw128(base + kQOff + (ks >> 2) * kHalf + cb, 16, 1024),
+                        tc05::smem_desc_sw128(kbase + (ks >> 2) * kHalfKV + cb, 16, 1024), idesc_qk, ks > 0);
+        }
+        tc05::commit(B(kSFull0 + st));
+        return true;
+      };
+      ok = mbar_wait_bounded(B(kQFull), 0, deadline) && issue_qk(0);
+      for (int j = 0; j < nkb && ok; ++j) {
+        if (j + 1 < nkb && !issue_qk(j + 1)) {  // S buffer (j+1)&1 was read by softmax(j-1): p_full(j-1) seen
           ok = false;
           break;
         }
-        tc05::fence_after_sync();
-        const uint32_t kbase = base + kStageOff + st * 2 * kTile, vbase = kbase + kTile;
-        // S = Q K^T: 8 k-steps of 16 along d (4 per 64-element half, 32 bytes apart).
-#pragma unroll
-        for (int ks = 0; ks < kD / 16; ++ks) {
-          const uint32_t off = (ks >> 2) * kHalf + (ks & 3) * 32;
-          tc05::mma_f16(tS, tc05::smem_desc_sw128(base + kQOff + off, 16, 1024),
-                        tc05::smem_desc_sw128(kbase + off, 16, 1024), idesc_qk, ks > 0);
-        }
-        tc05::commit(B(kSFull));
         if (!mbar_wait_bounded(B(kPFull), j & 1, deadline)) {
           ok = false;
           break;
         }
         tc05::fence_after_sync();
-        // O += P V: 8 k-steps of 16 keys; P K-major (halves of 64 keys), V MN-major (16 keys = 2048 B).
+        // O += P V: kKeys / 16 k-steps; P K-major (halves of 64 keys), V MN-major (16 keys = 2048 B).
+        const uint32_t vbase = base + kStageOff + (j & 1) * 2 * kTileKV + kTileKV;
 #pragma unroll
         for (int kt = 0; kt < kKeys / 16; ++kt) {
           const uint32_t poff = (kt >> 2) * kHalf + (kt & 3) * 32;
           tc05::mma_f16(tO, tc05::smem_desc_sw128(base + kPOff + poff, 16, 1024),
-                        tc05::smem_desc_sw128(vbase + kt * 2048, kHalf, 1024), idesc_pv, (j > 0 || kt > 0));
+                        tc05::smem_desc_sw128(vbase + kt * 2048, kHalfKV, 1024), idesc_pv, (j > 0 || kt > 0));
         }
         tc05::commit(B(kODone));
-        tc05::commit(B(kKvEmpty0 + st));
+        tc05::commit(B(kKvEmpty0 + (j & 1)));
       }
       tc05::commit(B(kAllDone));
       mbar_wait_bounded(B(kAllDone), 0, globaltimer_ns() + 1000000000ull);
@@ -179,32 +232,54 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
     const int r = threadIdx.x;  // 0..127, TMEM lane r
     const int R = tile * kRows + r;
     const bool valid = R < num_rows;
-    const int lim = valid ? start + R / G + 1 : 0;
+    // The row's visible keys, counted from key0: the causal diagonal, or the sequence's context
+    // clipped to the prefix (none of this chunk when it is shorter).
+    int lim = 0;
+    if (valid) {
+      if constexpr (kPrefix) {
+        lim = min(p.context_lens[R / G], p.prefix_tokens) - key0;
+        if (R % G == 0) {  // the sequence must map this chunk's pages to sequence 0's blocks
+          const int32_t* row = p.block_tables + static_cast<int64_t>(R / G) * p.bt_stride + key0 / 16;
+          bool mismatch = false;
+          for (int i = 0; i < npages; ++i) mismatch |= row[i] != bt[i];
+          if (mismatch) atomicOr(p.err, 16u);
+        }
+      } else {
+        lim = start + R / G + 1;
+      }
+    }
     const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
     const float sl2 = p.score_scale_log2;
-    float m = -INFINITY, l = 0.f;
+    float m = -INFINITY, l = 0.f;  // m: the reference P and l are taken against (lazily raised)
     for (int j = 0; j < nkb; ++j) {
-      const bool got = mbar_wait_bounded(B(kSFull), j & 1, deadline);
+      const bool got = mbar_wait_bounded(B(kSFull0 + (j & 1)), (j >> 1) & 1, deadline);
       if (!__all_sync(kFull, got)) {
         ok = false;
         break;
       }
       tc05::fence_after_sync();
       const int t0 = j * kKeys;
-      // Pass 1: the row's max over the block.
-      float mx = -INFINITY;
+      // The block's scores, scaled to log2 units (-inf past the row's limit), and their max.
+      float sv[kKeys];
 #pragma unroll
       for (int c = 0; c < kKeys / 32; ++c) {
         float v[32];
-        tc05::ld32(tS + lane_off + c * 32, v);
+        tc05::ld32(tS0 + (j & 1) * kKeys + lane_off + c * 32, v);
 #pragma unroll
-        for (int k = 0; k < 32; ++k)
-          if (t0 + c * 32 + k < lim) mx = fmaxf(mx, v[k] * sl2);
+        for (int k = 0; k < 32; ++k) sv[c * 32 + k] = t0 + c * 32 + k < lim ? v[k] * sl2 : -INFINITY;
       }
-      const float mn = fmaxf(m, mx);
-      const float ref = mn == -INFINITY ? 0.f : mn;
-      const float alpha = ex2(m - ref);
-      m = mn;
+      float mx = -INFINITY;
+#pragma unroll
+      for (int k = 0; k < kKeys; ++k) mx = fmaxf(mx, sv[k]);
+      // Raise the reference only when some row of the warp grew past it by more than 2^8.
+      const bool raise = __any_sync(kFull, mx > m + kLazyRescale);
+      float alpha = 1.f;
+      if (raise) {
+        const float mn = fmaxf(m, mx);
+        alpha = (m == -INFINITY || mn == -INFINITY) ? (m == -INFINITY ? 0.f : 1.f) : ex2(m - mn);
+        m = mn;
+      }
+      const float ref = m == -INFINITY ? 0.f : m;
       // P (and O's rescale) may only change once the previous P . V has finished.
       if (j > 0) {
         const bool done = mbar_wait_bounded(B(kODone), (j - 1) & 1, deadline);
@@ -213,20 +288,26 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
           break;
         }
         tc05::fence_after_sync();
+        if (raise) {
+#pragma unroll
+          for (int c = 0; c < kD / 32; ++c) {
+            float v[32];
+            tc05::ld32(tO + lane_off + c * 32, v);
+#pragma unroll
+            for (int k = 0; k < 32; ++k) v[k] *= alpha;
+            tc05::st32(tO + lane_off + c * 32, v);
+          }
+        }
       }
-      // Pass 2: P = 2^(s - ref) in 16-bit, row sums of the rounded values, into the swizzled P tile.
+      // P = 2^(s - ref) in 16-bit into the swizzled P tile; the row sum adds the rounded values.
       float rowsum = 0.f;
 #pragma unroll
       for (int c = 0; c < kKeys / 32; ++c) {
-        float v[32];
-        tc05::ld32(tS + lane_off + c * 32, v);
         uint32_t w[16];
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
-          const int t = t0 + c * 32 + 2 * k;
-          const float p0 = t < lim ? ex2(v[2 * k] * sl2 - ref) : 0.f;
-          const float p1 = t + 1 < lim ? ex2(v[2 * k + 1] * sl2 - ref) : 0.f;
-          w[k] = pack2<kBf16>(p0, p1);
+          const float s0 = sv[c * 32 + 2 * k], s1 = sv[c * 32 + 2 * k + 1];
+          w[k] = pack2<kBf16>(s0 == -INFINITY ? 0.f : ex2(s0 - ref), s1 == -INFINITY ? 0.f : ex2(s1 - ref));
           const float2 f = unpack2<kBf16>(w[k]);
           rowsum += f.x + f.y;
         }
@@ -241,17 +322,6 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         }
       }
       l = l * alpha + rowsum;
-      // Rescale O in TMEM when any row of the warp moved its max (j == 0: O is overwritten).
-      if (j > 0 && __any_sync(kFull, alpha != 1.f)) {
-#pragma unroll
-        for (int c = 0; c < kD / 32; ++c) {
-          float v[32];
-          tc05::ld32(tO + lane_off + c * 32, v);
-#pragma unroll
-          for (int k = 0; k < 32; ++k) v[k] *= alpha;
-          tc05::st32(tO + lane_off + c * 32, v);
-        }
-      }
       // Keys past every row's limit may hold any bits; zero those V rows so 0 * NaN cannot occur.
       if (t0 + kKeys > max_lim) {
         const bool landed = mbar_wait_bounded(B(kKvFull0 + (j & 1)), (j >> 1) & 1, deadline);
@@ -259,11 +329,11 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
           ok = false;
           break;
         }
-        const uint32_t vbase = base + kStageOff + (j & 1) * 2 * kTile + kTile;
-        const int first = max_lim - t0;  // rows [first, 128) of the V tile, both halves
+        const uint32_t vbase = base + kStageOff + (j & 1) * 2 * kTileKV + kTileKV;
+        const int first = max_lim - t0;  // rows [first, kKeys) of the V tile, both halves
         for (int idx = r; idx < (kKeys - first) * 16; idx += 128) {
           const int row = first + idx / 16, c16 = idx % 16;
-          asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(vbase + (c16 >> 3) * kHalf + row * 128 +
+          asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(vbase + (c16 >> 3) * kHalfKV + row * 128 +
                                                                          (c16 & 7) * 16),
                        "r"(0u)
                        : "memory");
@@ -274,11 +344,28 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
       __syncwarp();
       if (lane == 0) mbar_arrive(B(kPFull));
     }
-    // Epilogue: O / l -> out rows.
+    // Epilogue: O / l -> out rows, or (prefix) the row's (m, l, O) -> its workspace slot.
     if (ok) {
-      const bool done = mbar_wait_bounded(B(kODone), (nkb - 1) & 1, deadline);
-      if (__all_sync(kFull, done)) {
-        tc05::fence_after_sync();
+      const bool done = __all_sync(kFull, mbar_wait_bounded(B(kODone), (nkb - 1) & 1, deadline));
+      if (done) tc05::fence_after_sync();
+      if (!done) {
+        ok = false;
+      } else if constexpr (kPrefix) {
+        const int Hq = p.num_kv_heads * G;
+        const int64_t slot = (static_cast<int64_t>(valid ? R / G : 0) * Hq + hk * G + R % G) * p.ws_parts + s;
+        float* dst = p.ws_acc + slot * kD;
+#pragma unroll
+        for (int c = 0; c < kD / 32; ++c) {
+          float v[32];
+          tc05::ld32(tO + lane_off + c * 32, v);
+          if (valid) {
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+              *reinterpret_cast<float4*>(dst + c * 32 + 4 * q) = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+          }
+        }
+        if (valid) *reinterpret_cast<float2*>(p.ws_ml + slot * 2) = make_float2(m, l);
+      } else {
         const float inv = l > 0.f ? 1.f / l : 0.f;
         uint16_t* dst = static_cast<uint16_t*>(p.out) + static_cast<int64_t>(q_row0 + (valid ? R / G : 0)) * p.o_stride_t +
                         static_cast<int64_t>(hk * G + R % G) * p.o_stride_h;
@@ -298,19 +385,38 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             }
           }
         }
-      } else {
-        ok = false;
       }
     }
     if (!ok && lane == 0) atomicOr(p.err, 4u);
   }
-  pdl_launch_dependents();
+  if constexpr (!kPrefix) pdl_launch_dependents();
   tc05::fence_before_sync();
   __syncthreads();
   if (warp == 5) {
     tc05::fence_after_sync();
     tc05::dealloc(tmem, 256);
   }
+}
+
+template <bool kBf16, bool kPrefix>
+cudaError_t launch_tc(dim3 grid, const CUtensorMap& qm, const CUtensorMap& km, const CUtensorMap& vm, const MqParams& p,
+                      cudaStream_t st) {
+  constexpr int kKeys = PA_PREFILL_TC_KEYS;
+  using C = TcCfg<kKeys>;
+  auto kern = prefill_tc_kernel<kBf16, kKeys, kPrefix>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, qm, km, vm, p);
 }
 
 }  // namespace
@@ -322,21 +428,22 @@ bool prefill_tc_supported(int head_dim, int group) {
 cudaError_t launch_prefill_tc(KvType kv, const CUtensorMap& qm, const CUtensorMap& km, const CUtensorMap& vm,
                               const MqParams& p, int max_query_len, cudaStream_t st) {
   if (kv != KvType::F16 && kv != KvType::BF16) return cudaErrorInvalidValue;
-  auto kern = kv == KvType::BF16 ? prefill_tc_kernel<true> : prefill_tc_kernel<false>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-  if (e != cudaSuccess) return e;
   const int64_t rows = static_cast<int64_t>(max_query_len) * p.group;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>((rows + kRows - 1) / kRows), p.num_kv_heads, p.num_seqs);
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = kSmemBytes;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, qm, km, vm, p);
+  const dim3 grid(static_cast<unsigned>((rows + kRows - 1) / kRows), p.num_kv_heads, p.num_seqs);
+  return kv == KvType::BF16 ? launch_tc<true, false>(grid, qm, km, vm, p, st)
+                            : launch_tc<false, false>(grid, qm, km, vm, p, st);
+}
+
+// Shared-prefix mode: grid (row tiles of num_seqs * G, KV heads, prefix chunks); chunk_tokens must be
+// a multiple of the key block.
+cudaError_t launch_prefix_tc(KvType kv, const CUtensorMap& qm, const CUtensorMap& km, const CUtensorMap& vm,
+                             const MqParams& p, cudaStream_t st) {
+  if (kv != KvType::F16 && kv != KvType::BF16) return cudaErrorInvalidValue;
+  if (p.chunk_tokens <= 0 || p.chunk_tokens % PA_PREFILL_TC_KEYS || p.prefix_tokens % 16) return cudaErrorInvalidValue;
+  const int64_t rows = static_cast<int64_t>(p.num_seqs) * p.group;
+  const dim3 grid(static_cast<unsigned>((rows + kRows - 1) / kRows), p.num_kv_heads, p.num_chunks);
+  return kv == KvType::BF16 ? launch_tc<true, true>(grid, qm, km, vm, p, st)
+                            : launch_tc<false, true>(grid, qm, km, vm, p, st);
 }
 
 }  // namespace pa

@@ -125,7 +125,7 @@ class DeviceCase:
         return out
 
     def cascade(self, fused: bool = True, partition_tokens: int = 0, out: Optional[torch.Tensor] = None,
-                error_word: Optional[torch.Tensor] = None) -> torch.Tensor:
+                error_word: Optional[torch.Tensor] = None, prefix_kernel: int = -1) -> torch.Tensor:
         """pa_decode_cascade over the workload's shared prefix (with the new-token write if fused)."""
         w = self.w
         out = self.out if out is None else out
@@ -135,7 +135,8 @@ class DeviceCase:
         nk = (self.new_k, self.new_v, self.new_slots) if fused else (None, None, None)
         pa.pa_decode_cascade(out, self.q, *nk, self.k_cache, self.v_cache, self.bt, self.lens,
                              w.shared_prefix_tokens, w.scale, w.num_kv_heads, max_context_len=self.max_ctx,
-                             partition_tokens=partition_tokens, workspace=ws, error_word=error_word)
+                             partition_tokens=partition_tokens, workspace=ws, error_word=error_word,
+                             prefix_kernel=prefix_kernel)
         return out
 
     def pool_bytes(self):

@@ -1,8 +1,9 @@
 """GPU parity of shared-prefix (cascade) decode against the float64 oracle.
 
 pa_decode_cascade reads the prefix every sequence shares once per KV head (all B * G query rows as
-one tensor-core contraction), the rest of each context with the decode kernel, and merges the two
-softmax partials; the oracle is the plain definition over each sequence's whole context.
+one tensor-core contraction, by the tcgen05 kernel or the warp-level mma kernel), the rest of each
+context with the decode kernel, and merges the two softmax partials; the oracle is the plain
+definition over each sequence's whole context.
 """
 import numpy as np
 import pytest
@@ -20,8 +21,12 @@ def max_err(got, want):
     return float(np.max(np.abs(got.double().cpu().numpy() - want)))
 
 
+PREFIX_KERNELS = [0, 1]  # warp-level mma, tcgen05
+
+
+@pytest.mark.parametrize("prefix_kernel", PREFIX_KERNELS)
 @pytest.mark.parametrize("fused", [True, False])
-def test_cascade_matches_oracle(fused):
+def test_cascade_matches_oracle(fused, prefix_kernel):
     w = W.ALL["prefix_gqa_small"]
     case = oracle_case.build(w)
     want = oracle_case.expected_out(case)
@@ -29,7 +34,7 @@ def test_cascade_matches_oracle(fused):
     if not fused:
         dev.write_new_token()
     for pt in (0, 16, 48):
-        out = dev.cascade(fused=fused, partition_tokens=pt)
+        out = dev.cascade(fused=fused, partition_tokens=pt, prefix_kernel=prefix_kernel)
         torch.cuda.synchronize()
         assert max_err(out, want) <= TOL[w.kv_dtype], pt
     assert pa.pa_read_device_error(clear=True) == 0
@@ -42,13 +47,63 @@ def test_cascade_equals_plain_decode_within_rounding():
     dev = DeviceCase(w)
     dev.write_new_token()
     a = dev.decode(kernel=1).clone()
-    b = dev.cascade(fused=False).clone()
+    b = dev.cascade(fused=False, prefix_kernel=0).clone()
+    c = dev.cascade(fused=False, prefix_kernel=1).clone()
     torch.cuda.synchronize()
     assert (a.double() - b.double()).abs().max().item() <= TOL[w.kv_dtype]
+    assert (c.double() - b.double()).abs().max().item() <= TOL[w.kv_dtype]
 
 
+def _shared_prefix_case(lens, hq, hkv, prefix, dtype, seed, nb_extra=0):
+    """Block tables whose first prefix / 16 entries are blocks 0 .. prefix / 16 - 1 in every row."""
+    B, D = len(lens), 128
+    g = torch.Generator().manual_seed(seed)
+    width = max(-(-max(lens) // 16), prefix // 16)
+    own = sum(max(0, -(-n // 16) - prefix // 16) for n in lens)
+    nb = prefix // 16 + own + nb_extra
+    bt = torch.full((B, width), -1, dtype=torch.int32)
+    order = (torch.randperm(own, generator=g) + prefix // 16).tolist()
+    for s, n in enumerate(lens):
+        for j in range(max(-(-n // 16), prefix // 16)):  # shorter sequences still list the prefix blocks
+            bt[s, j] = j if j < prefix // 16 else order.pop()
+    kc = torch.randn(nb, hkv, 16, D, generator=g).to(dtype)
+    vc = torch.randn(nb, hkv, 16, D, generator=g).to(dtype)
+    q = torch.randn(B, hq, D, generator=g).to(dtype)
+    return q, kc, vc, bt
+
+
+def _oracle_out(q, kc, vc, bt, lens, scale, hkv, kv):
+    from oracle import attention
+    nb, D = kc.shape[0], kc.shape[3]
+    kb = kc.view(torch.int16).numpy().view(np.uint8).reshape(nb, hkv, 16, D * 2)
+    vb = vc.view(torch.int16).numpy().view(np.uint8).reshape(nb, hkv, 16, D * 2)
+    return attention.decode_paged(q.double().numpy(), kb, vb, bt.numpy(), lens, scale, hkv, kv)
+
+
+@pytest.mark.parametrize("prefix_kernel", PREFIX_KERNELS)
+@pytest.mark.parametrize("dtype,kv", [(torch.bfloat16, "bf16"), (torch.float16, "f16")])
+def test_cascade_prefix_of_several_chunks(prefix_kernel, dtype, kv):
+    """A 640-token prefix: two full 256-token chunks and a ragged one; 40 sequences x 4 group heads
+    (two 128-row tiles, the second ragged); some contexts end inside the prefix, one exactly at it."""
+    rng = np.random.default_rng(7)
+    lens = [int(x) for x in 640 + rng.integers(1, 120, 40)]
+    lens[3], lens[17], lens[30], lens[39] = 300, 640, 17, 641
+    q, kc, vc, bt = _shared_prefix_case(lens, 8, 2, 640, dtype, seed=640)
+    n = pa.pa_decode_cascade_workspace_bytes(len(lens), 8, 2, 128, max(lens), 640, 0)
+    ws = torch.empty(n, dtype=torch.uint8, device="cuda")
+    out = torch.empty(len(lens), 8, 128, dtype=dtype, device="cuda")
+    pa.pa_decode_cascade(out, q.cuda(), None, None, None, kc.cuda(), vc.cuda(), bt.cuda(),
+                         torch.tensor(lens, dtype=torch.int32).cuda(), 640, 0.0884, 2, workspace=ws,
+                         max_context_len=max(lens), prefix_kernel=prefix_kernel)
+    torch.cuda.synchronize()
+    assert pa.pa_read_device_error(clear=True) == 0
+    want = _oracle_out(q, kc, vc, bt, lens, 0.0884, 2, kv)
+    assert max_err(out, want) <= TOL[kv]
+
+
+@pytest.mark.parametrize("prefix_kernel", PREFIX_KERNELS)
 @pytest.mark.parametrize("lens", [(5, 64, 100, 16, 129, 40), (64, 64, 65, 200, 1, 33)])
-def test_cascade_with_sequences_shorter_than_the_prefix(lens):
+def test_cascade_with_sequences_shorter_than_the_prefix(lens, prefix_kernel):
     """Rows stop at their own context even inside the shared prefix; f16, G = 1 and G = 8 heads."""
     from oracle import attention
     for hq, hkv in ((4, 4), (16, 2)):
@@ -75,7 +130,7 @@ def test_cascade_with_sequences_shorter_than_the_prefix(lens):
         ws = torch.empty(n, dtype=torch.uint8, device="cuda")
         out = torch.empty(B, hq, D, dtype=torch.float16, device="cuda")
         pa.pa_decode_cascade(out, q.cuda(), None, None, None, kc.cuda(), vc.cuda(), bt.cuda(), lens_t.cuda(), P,
-                             0.088, hkv, workspace=ws)
+                             0.088, hkv, workspace=ws, prefix_kernel=prefix_kernel)
         torch.cuda.synchronize()
         assert pa.pa_read_device_error(clear=True) == 0
         kb = kc.view(torch.int16).numpy().view(np.uint8).reshape(nb, hkv, 16, D * 2)
@@ -84,7 +139,8 @@ def test_cascade_with_sequences_shorter_than_the_prefix(lens):
         assert max_err(out, want) <= TOL["f16"]
 
 
-def test_cascade_reports_a_table_without_the_shared_prefix():
+@pytest.mark.parametrize("prefix_kernel", PREFIX_KERNELS)
+def test_cascade_reports_a_table_without_the_shared_prefix(prefix_kernel):
     w = W.ALL["prefix_gqa_small"]
     dev = DeviceCase(w)
     dev.write_new_token()
@@ -93,17 +149,18 @@ def test_cascade_reports_a_table_without_the_shared_prefix():
     bt[2, 1] = int(bt[0, 1]) + 1 if int(bt[0, 1]) + 1 < w.num_blocks else 0
     old = dev.bt
     dev.bt = bt
-    dev.cascade(fused=False, error_word=word)
+    dev.cascade(fused=False, error_word=word, prefix_kernel=prefix_kernel)
     torch.cuda.synchronize()
     dev.bt = old
     assert int(word.item()) & pa.PA_DEVERR_PREFIX
 
 
-def test_full_size_prefix_workload_sampled():
+@pytest.mark.parametrize("prefix_kernel", PREFIX_KERNELS)
+def test_full_size_prefix_workload_sampled(prefix_kernel):
     from oracle import attention
     w = W.FULL["prefix_gqa"]
     dev = DeviceCase(w, sentinel=False)
-    out = dev.cascade(fused=True).cpu()
+    out = dev.cascade(fused=True, prefix_kernel=prefix_kernel).cpu()
     assert pa.pa_read_device_error(clear=True) == 0
     lens = dev.lens_host
     rng = np.random.default_rng(11)
