@@ -8,22 +8,20 @@
 //   one chunk of the prefix pages every block table shares and writes the rows' partial softmax
 //   state (m, l, unnormalised acc) to the split workspace, merged later with the sequence's suffix.
 //
-// CTA = 128 query rows of one KV head. Per block of KEYS keys (KEYS / 16 pages), with the block's K
-// and V staged by TMA in 128-byte-swizzled shared memory:
-//   S[128 x KEYS] = Q . K^T     tcgen05.mma kind::f16, A = Q (K-major), B = K (K-major), D in TMEM
+// CTA = 128 query rows of one KV head, two CTAs per SM (one's softmax overlaps the other's MMAs).
+// Per block of 64 keys (4 pages), with the block's K and V staged by TMA in 128-byte-swizzled
+// shared memory:
+//   S[128 x 64] = Q . K^T       tcgen05.mma kind::f16, A = Q (K-major), B = K (K-major), D in TMEM;
+//                               two S buffers, so QK of the next block runs during this softmax
 //   softmax                     4 warps, one row per thread, S read from TMEM (tcgen05.ld), running
-//                               max / sum in registers, P written (bf16/f16) to shared memory, O
-//                               rescaled in TMEM when a row's max moved
-//   O[128 x 128] += P . V       A = P (K-major), B = V (MN-major: d contiguous), D in TMEM
+//                               max / sum in registers, P (bf16/f16) written back to TMEM over S,
+//                               O rescaled in TMEM only when a row's max grew past the lazy bound
+//   O[128 x 128] += P . V       A = P from TMEM, B = V (MN-major: d contiguous), D in TMEM
 // Warps: 0-3 softmax + epilogue, 4 TMA producer (Q once, then K/V blocks into a 2-stage ring),
 // 5 MMA issuer (one thread) and TMEM owner. Every mbarrier wait is bounded.
 #include "internal.h"
 #include "pa_device.cuh"
 #include "tc05.cuh"
-
-#ifndef PA_PREFILL_TC_KEYS
-#define PA_PREFILL_TC_KEYS 64
-#endif
 
 namespace pa {
 namespace {
@@ -34,33 +32,36 @@ constexpr int kThreads = 192;
 constexpr uint32_t kHalf = 16384;  // one 64-element (128-byte) column half of a 128-row tile
 constexpr uint32_t kTile = 2 * kHalf;
 
-// KEYS keys per block: 128 (one CTA per SM, 2 stages of 64 KB) or 64 (two CTAs per SM sharing the
-// tensor core, so one CTA's softmax overlaps the other's MMAs: 112 KB of shared memory each).
-template <int KEYS>
-struct TcCfg {
-  static constexpr uint32_t kHalfKV = KEYS * 128;            // a 64-element column half of a K or V tile
-  static constexpr uint32_t kTileKV = 2 * kHalfKV;
-  static constexpr uint32_t kQOff = 0;
-  static constexpr uint32_t kStageOff = kTile;                // stage s: K at + s * 2 * kTileKV, V after it
-  static constexpr uint32_t kPOff = kStageOff + 4 * kTileKV;  // P tile: KEYS / 64 halves of 128 x 128 B
-  static constexpr uint32_t kBarOff = kPOff + (KEYS / 64) * kHalf;
-  static constexpr uint32_t kSmemBytes = kBarOff + 128;
-  static constexpr int kMinBlocks = KEYS == 64 ? 2 : 1;
-};
+// Shared memory (96 KB + barriers): Q tile, then two stages of (K tile, V tile) of 64 keys each.
+constexpr int kKeys = 64;
+constexpr uint32_t kHalfKV = kKeys * 128;  // a 64-element column half of a K or V tile
+constexpr uint32_t kTileKV = 2 * kHalfKV;
+constexpr uint32_t kQOff = 0;
+constexpr uint32_t kStageOff = kTile;      // stage s: K at + s * 2 * kTileKV, V after it
+constexpr uint32_t kBarOff = kStageOff + 4 * kTileKV;
+constexpr uint32_t kSmemBytes = kBarOff + 128;
+// TMEM: two S buffers of kKeys columns, then O's 128 columns.
+constexpr uint32_t kTmemCols = 256;
+static_assert(2 * kKeys + kD <= kTmemCols, "S buffers and O must fit the allocation");
 // barrier slots (8 bytes each)
 enum { kQFull = 0, kKvFull0 = 1, kKvEmpty0 = 3, kSFull0 = 5, kPFull = 7, kODone = 8, kAllDone = 9, kTmemSlot = 10 };
 // O is rescaled only when a row's running max grows by more than this (log2 units); until then P and
 // the row sum keep the older reference, so the result is unchanged and P stays below 2^8.
 constexpr float kLazyRescale = 8.f;
 
-template <bool kBf16, int KEYS, bool kPrefix>
-__global__ void __launch_bounds__(kThreads, TcCfg<KEYS>::kMinBlocks)
+// Max (kMax) or min of n values in four independent chains.
+template <bool kMax, int n>
+__device__ __forceinline__ float extreme(const float (&v)[n]) {
+  float e[4] = {v[0], v[1], v[2], v[3]};
+#pragma unroll
+  for (int k = 4; k < n; ++k) e[k & 3] = kMax ? fmaxf(e[k & 3], v[k]) : fminf(e[k & 3], v[k]);
+  return kMax ? fmaxf(fmaxf(e[0], e[1]), fmaxf(e[2], e[3])) : fminf(fminf(e[0], e[1]), fminf(e[2], e[3]));
+}
+
+template <bool kBf16, bool kPrefix>
+__global__ void __launch_bounds__(kThreads, 2)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
                       const __grid_constant__ CUtensorMap vmap, const MqParams p) {
-  using C = TcCfg<KEYS>;
-  constexpr int kKeys = KEYS;
-  constexpr uint32_t kHalfKV = C::kHalfKV, kTileKV = C::kTileKV, kQOff = C::kQOff, kStageOff = C::kStageOff;
-  constexpr uint32_t kPOff = C::kPOff, kBarOff = C::kBarOff;
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t base = smem_u32(smem);
   if (base & 1023u) {  // the swizzled tiles need 1024-byte alignment; never seen, but do not guess
@@ -124,9 +125,6 @@ __global__ void __launch_bounds__(kThreads, TcCfg<KEYS>::kMinBlocks)
     mbar_init(B(kAllDone), 1);
     fence_barrier_init();
   }
-  // TMEM: two S buffers of kKeys columns (QK of the next block runs while this one's softmax does),
-  // then O's 128 columns.
-  constexpr uint32_t kTmemCols = 2 * kKeys + kD <= 256 ? 256 : 512;
   if (warp == 5) tc05::alloc(B(kTmemSlot), kTmemCols);
   tc05::fence_before_sync();
   __syncthreads();
@@ -138,6 +136,18 @@ __global__ void __launch_bounds__(kThreads, TcCfg<KEYS>::kMinBlocks)
 
   if (warp == 4) {
     // ---- producer -------------------------------------------------------------------------------
+    if constexpr (kPrefix) {
+      if (lane > 0) {
+        // Lanes 1-31: every sequence of the tile must map this chunk's pages to sequence 0's blocks.
+        const int s0 = tile * kRows / G, s1 = min((tile + 1) * kRows, num_rows) / G;  // [s0, s1)
+        bool mismatch = false;
+        for (int idx = lane - 1; idx < (s1 - s0) * npages; idx += 31) {
+          const int sq = s0 + idx / npages, i = idx % npages;
+          mismatch |= p.block_tables[static_cast<int64_t>(sq) * p.bt_stride + key0 / 16 + i] != bt[i];
+        }
+        if (mismatch) atomicOr(p.err, 16u);
+      }
+    }
     if (lane == 0) {
       prefetch_tensormap(&qmap);
       mbar_arrive_expect_tx(B(kQFull), kTile);
@@ -203,22 +213,27 @@ __global__ void __launch_bounds__(kThreads, TcCfg<KEYS>::kMinBlocks)
       };
       ok = mbar_wait_bounded(B(kQFull), 0, deadline) && issue_qk(0);
       for (int j = 0; j < nkb && ok; ++j) {
-        if (j + 1 < nkb && !issue_qk(j + 1)) {  // S buffer (j+1)&1 was read by softmax(j-1): p_full(j-1) seen
-          ok = false;
-          break;
+        // S(j+1) goes to the buffer that holds P(j-1): softmax(j-1) is done with it (p_full(j-1) was
+        // seen), but P(j-1) . V may still be reading it, so wait for that MMA to finish first.
+        if (j + 1 < nkb) {
+          if ((j > 0 && !mbar_wait_bounded(B(kODone), (j - 1) & 1, deadline)) || !issue_qk(j + 1)) {
+            ok = false;
+            break;
+          }
         }
         if (!mbar_wait_bounded(B(kPFull), j & 1, deadline)) {
           ok = false;
           break;
         }
         tc05::fence_after_sync();
-        // O += P V: kKeys / 16 k-steps; P K-major (halves of 64 keys), V MN-major (16 keys = 2048 B).
+        // O += P V: kKeys / 16 k-steps; P from TMEM (written over S(j), 8 columns = 16 keys per step),
+        // V MN-major in shared memory (16 keys = 2048 B). The next QK into this S buffer is issued
+        // after these MMAs by this thread, and MMAs from one thread execute in order.
         const uint32_t vbase = base + kStageOff + (j & 1) * 2 * kTileKV + kTileKV;
 #pragma unroll
         for (int kt = 0; kt < kKeys / 16; ++kt) {
-          const uint32_t poff = (kt >> 2) * kHalf + (kt & 3) * 32;
-          tc05::mma_f16(tO, tc05::smem_desc_sw128(base + kPOff + poff, 16, 1024),
-                        tc05::smem_desc_sw128(vbase + kt * 2048, kHalfKV, 1024), idesc_pv, (j > 0 || kt > 0));
+          tc05::mma_f16_ts(tO, tS0 + (j & 1) * kKeys + kt * 8, tc05::smem_desc_sw128(vbase + kt * 2048, kHalfKV, 1024),
+                           idesc_pv, (j > 0 || kt > 0));
         }
         tc05::commit(B(kODone));
         tc05::commit(B(kKvEmpty0 + (j & 1)));
@@ -238,12 +253,6 @@ __global__ void __launch_bounds__(kThreads, TcCfg<KEYS>::kMinBlocks)
     if (valid) {
       if constexpr (kPrefix) {
         lim = min(p.context_lens[R / G], p.prefix_tokens) - key0;
-        if (R % G == 0) {  // the sequence must map this chunk's pages to sequence 0's blocks
-          const int32_t* row = p.block_tables + static_cast<int64_t>(R / G) * p.bt_stride + key0 / 16;
-          bool mismatch = false;
-          for (int i = 0; i < npages; ++i) mismatch |= row[i] != bt[i];
-          if (mismatch) atomicOr(p.err, 16u);
-        }
       } else {
         lim = start + R / G + 1;
       }
@@ -259,18 +268,23 @@ __global__ void __launch_bounds__(kThreads, TcCfg<KEYS>::kMinBlocks)
       }
       tc05::fence_after_sync();
       const int t0 = j * kKeys;
-      // The block's scores, scaled to log2 units (-inf past the row's limit), and their max.
+      // The block's scores and their max in log2 units. Blocks where no row of the warp reaches its
+      // limit keep raw scores (the scale is applied in the exponent's FMA; the max of the scaled
+      // scores is the raw max times a positive scale, the raw min times a negative one); blocks
+      // that reach a limit are scaled here and the keys past it set to -inf.
       float sv[kKeys];
+      tc05::ld64(tS0 + (j & 1) * kKeys + lane_off, sv);
+      float mul = sl2, mx;
+      if (__any_sync(kFull, t0 + kKeys > lim)) {
 #pragma unroll
-      for (int c = 0; c < kKeys / 32; ++c) {
-        float v[32];
-        tc05::ld32(tS0 + (j & 1) * kKeys + lane_off + c * 32, v);
-#pragma unroll
-        for (int k = 0; k < 32; ++k) sv[c * 32 + k] = t0 + c * 32 + k < lim ? v[k] * sl2 : -INFINITY;
+        for (int k = 0; k < kKeys; ++k) sv[k] = t0 + k < lim ? sv[k] * sl2 : -INFINITY;
+        mul = 1.f;
+        mx = extreme<true, kKeys>(sv);
+      } else if (sl2 >= 0.f) {
+        mx = extreme<true, kKeys>(sv) * sl2;
+      } else {
+        mx = extreme<false, kKeys>(sv) * sl2;
       }
-      float mx = -INFINITY;
-#pragma unroll
-      for (int k = 0; k < kKeys; ++k) mx = fmaxf(mx, sv[k]);
       // Raise the reference only when some row of the warp grew past it by more than 2^8.
       const bool raise = __any_sync(kFull, mx > m + kLazyRescale);
       float alpha = 1.f;
@@ -279,49 +293,40 @@ __global__ void __launch_bounds__(kThreads, TcCfg<KEYS>::kMinBlocks)
         alpha = (m == -INFINITY || mn == -INFINITY) ? (m == -INFINITY ? 0.f : 1.f) : ex2(m - mn);
         m = mn;
       }
-      const float ref = m == -INFINITY ? 0.f : m;
-      // P (and O's rescale) may only change once the previous P . V has finished.
-      if (j > 0) {
+      const float nref = m == -INFINITY ? 0.f : -m;
+      // P = 2^(s * scale - ref) (ex2 of -inf is +0) in 16-bit, packed two keys per word; the row
+      // sum adds the float values in four chains.
+      uint32_t w[kKeys / 2];
+      float rs[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int k = 0; k < kKeys / 2; ++k) {
+        const float p0 = ex2(fmaf(sv[2 * k], mul, nref));
+        const float p1 = ex2(fmaf(sv[2 * k + 1], mul, nref));
+        w[k] = pack2<kBf16>(p0, p1);
+        rs[(2 * k) & 3] += p0;
+        rs[(2 * k + 1) & 3] += p1;
+      }
+      l = l * alpha + ((rs[0] + rs[1]) + (rs[2] + rs[3]));
+      // O's rescale waits for the previous P . V (only when the reference moved).
+      if (raise && j > 0) {
         const bool done = mbar_wait_bounded(B(kODone), (j - 1) & 1, deadline);
         if (!__all_sync(kFull, done)) {
           ok = false;
           break;
         }
         tc05::fence_after_sync();
-        if (raise) {
 #pragma unroll
-          for (int c = 0; c < kD / 32; ++c) {
-            float v[32];
-            tc05::ld32(tO + lane_off + c * 32, v);
+        for (int c = 0; c < kD / 32; ++c) {
+          float v[32];
+          tc05::ld32(tO + lane_off + c * 32, v);
 #pragma unroll
-            for (int k = 0; k < 32; ++k) v[k] *= alpha;
-            tc05::st32(tO + lane_off + c * 32, v);
-          }
+          for (int k = 0; k < 32; ++k) v[k] *= alpha;
+          tc05::st32(tO + lane_off + c * 32, v);
         }
       }
-      // P = 2^(s - ref) in 16-bit into the swizzled P tile; the row sum adds the rounded values.
-      float rowsum = 0.f;
-#pragma unroll
-      for (int c = 0; c < kKeys / 32; ++c) {
-        uint32_t w[16];
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          const float s0 = sv[c * 32 + 2 * k], s1 = sv[c * 32 + 2 * k + 1];
-          w[k] = pack2<kBf16>(s0 == -INFINITY ? 0.f : ex2(s0 - ref), s1 == -INFINITY ? 0.f : ex2(s1 - ref));
-          const float2 f = unpack2<kBf16>(w[k]);
-          rowsum += f.x + f.y;
-        }
-        // 32 keys = 64 bytes = 4 chunks of the row, in key half (c >> 1), chunks (c & 1) * 4 + q.
-        const uint32_t row = base + kPOff + (c >> 1) * kHalf + r * 128;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const uint32_t chunk = ((c & 1) * 4 + q) ^ (r & 7);
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row + chunk * 16), "r"(w[4 * q]),
-                       "r"(w[4 * q + 1]), "r"(w[4 * q + 2]), "r"(w[4 * q + 3])
-                       : "memory");
-        }
-      }
-      l = l * alpha + rowsum;
+      // P over the first kKeys / 2 columns of S(j) (whose scores are all in registers by now).
+      static_assert(kKeys / 2 == 32, "P is stored as one 32-column TMEM store");
+      tc05::st32u(tS0 + (j & 1) * kKeys + lane_off, w);
       // Keys past every row's limit may hold any bits; zero those V rows so 0 * NaN cannot occur.
       if (t0 + kKeys > max_lim) {
         const bool landed = mbar_wait_bounded(B(kKvFull0 + (j & 1)), (j >> 1) & 1, deadline);
@@ -338,8 +343,8 @@ __global__ void __launch_bounds__(kThreads, TcCfg<KEYS>::kMinBlocks)
                        "r"(0u)
                        : "memory");
         }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       }
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       tc05::fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(B(kPFull));
@@ -394,22 +399,20 @@ __global__ void __launch_bounds__(kThreads, TcCfg<KEYS>::kMinBlocks)
   __syncthreads();
   if (warp == 5) {
     tc05::fence_after_sync();
-    tc05::dealloc(tmem, 256);
+    tc05::dealloc(tmem, kTmemCols);
   }
 }
 
 template <bool kBf16, bool kPrefix>
 cudaError_t launch_tc(dim3 grid, const CUtensorMap& qm, const CUtensorMap& km, const CUtensorMap& vm, const MqParams& p,
                       cudaStream_t st) {
-  constexpr int kKeys = PA_PREFILL_TC_KEYS;
-  using C = TcCfg<kKeys>;
-  auto kern = prefill_tc_kernel<kBf16, kKeys, kPrefix>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  auto kern = prefill_tc_kernel<kBf16, kPrefix>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.dynamicSmemBytes = kSmemBytes;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -439,7 +442,7 @@ cudaError_t launch_prefill_tc(KvType kv, const CUtensorMap& qm, const CUtensorMa
 cudaError_t launch_prefix_tc(KvType kv, const CUtensorMap& qm, const CUtensorMap& km, const CUtensorMap& vm,
                              const MqParams& p, cudaStream_t st) {
   if (kv != KvType::F16 && kv != KvType::BF16) return cudaErrorInvalidValue;
-  if (p.chunk_tokens <= 0 || p.chunk_tokens % PA_PREFILL_TC_KEYS || p.prefix_tokens % 16) return cudaErrorInvalidValue;
+  if (p.chunk_tokens <= 0 || p.chunk_tokens % kKeys || p.prefix_tokens % 16) return cudaErrorInvalidValue;
   const int64_t rows = static_cast<int64_t>(p.num_seqs) * p.group;
   const dim3 grid(static_cast<unsigned>((rows + kRows - 1) / kRows), p.num_kv_heads, p.num_chunks);
   return kv == KvType::BF16 ? launch_tc<true, true>(grid, qm, km, vm, p, st)

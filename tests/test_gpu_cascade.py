@@ -50,8 +50,9 @@ def test_cascade_equals_plain_decode_within_rounding():
     b = dev.cascade(fused=False, prefix_kernel=0).clone()
     c = dev.cascade(fused=False, prefix_kernel=1).clone()
     torch.cuda.synchronize()
-    assert (a.double() - b.double()).abs().max().item() <= TOL[w.kv_dtype]
-    assert (c.double() - b.double()).abs().max().item() <= TOL[w.kv_dtype]
+    # Each is within TOL of the exact result, so two of them differ by at most 2 * TOL.
+    assert (a.double() - b.double()).abs().max().item() <= 2 * TOL[w.kv_dtype]
+    assert (c.double() - b.double()).abs().max().item() <= 2 * TOL[w.kv_dtype]
 
 
 def _shared_prefix_case(lens, hq, hkv, prefix, dtype, seed, nb_extra=0):
