@@ -17,8 +17,8 @@
 //                               max / sum in registers, P (bf16/f16) written back to TMEM over S,
 //                               O rescaled in TMEM only when a row's max grew past the lazy bound
 //   O[128 x 128] += P . V       A = P from TMEM, B = V (MN-major: d contiguous), D in TMEM
-// Warps: 0-3 softmax + epilogue, 4 TMA producer (Q once, then K/V blocks into a 2-stage ring),
-// 5 MMA issuer (one thread) and TMEM owner. Every mbarrier wait is bounded.
+// Warps: 0-3 softmax + epilogue, 4 TMA producer of Q and K (3-stage ring), 5 MMA issuer (one
+// thread) and TMEM owner, 6 TMA producer of V (2-stage ring). Every mbarrier wait is bounded.
 #include "internal.h"
 #include "pa_device.cuh"
 #include "tc05.cuh"
@@ -28,23 +28,39 @@ namespace {
 
 constexpr int kD = 128;
 constexpr int kRows = 128;   // query rows per CTA
-constexpr int kThreads = 192;
+constexpr int kThreads = 224;
 constexpr uint32_t kHalf = 16384;  // one 64-element (128-byte) column half of a 128-row tile
 constexpr uint32_t kTile = 2 * kHalf;
 
-// Shared memory (96 KB + barriers): Q tile, then two stages of (K tile, V tile) of 64 keys each.
+// Shared memory (112 KB + barriers): the Q tile, three stages of K tiles and two of V tiles, 64 keys
+// each. K and V rings are separate: a K stage frees when its QK has run, long before the block's P.V,
+// so the K copies of block j + 2 are in flight while block j is still being processed.
 constexpr int kKeys = 64;
+constexpr int kKStages = 3, kVStages = 2;
 constexpr uint32_t kHalfKV = kKeys * 128;  // a 64-element column half of a K or V tile
 constexpr uint32_t kTileKV = 2 * kHalfKV;
 constexpr uint32_t kQOff = 0;
-constexpr uint32_t kStageOff = kTile;      // stage s: K at + s * 2 * kTileKV, V after it
-constexpr uint32_t kBarOff = kStageOff + 4 * kTileKV;
-constexpr uint32_t kSmemBytes = kBarOff + 128;
+constexpr uint32_t kKOff = kTile;
+constexpr uint32_t kVOff = kKOff + kKStages * kTileKV;
+constexpr uint32_t kBarOff = kVOff + kVStages * kTileKV;
+constexpr uint32_t kSmemBytes = kBarOff + 256;
 // TMEM: two S buffers of kKeys columns, then O's 128 columns.
 constexpr uint32_t kTmemCols = 256;
 static_assert(2 * kKeys + kD <= kTmemCols, "S buffers and O must fit the allocation");
 // barrier slots (8 bytes each)
-enum { kQFull = 0, kKvFull0 = 1, kKvEmpty0 = 3, kSFull0 = 5, kPFull = 7, kODone = 8, kAllDone = 9, kTmemSlot = 10 };
+enum {
+  kQFull = 0,
+  kKFull0 = 1,   // kKStages
+  kKEmpty0 = 4,  // kKStages
+  kVFull0 = 7,   // kVStages
+  kVEmpty0 = 9,  // kVStages
+  kSFull0 = 11,  // 2
+  kPFull = 13,
+  kODone = 14,
+  kAllDone = 15,
+  kTmemSlot = 16,
+};
+static_assert(8 * (kTmemSlot + 1) <= 256, "barrier area");
 // O is rescaled only when a row's running max grows by more than this (log2 units); until then P and
 // the row sum keep the older reference, so the result is unchanged and P stays below 2^8.
 constexpr float kLazyRescale = 8.f;
@@ -114,10 +130,14 @@ __global__ void __launch_bounds__(kThreads, 2)
 
   if (threadIdx.x == 0) {
     mbar_init(B(kQFull), 1);
-    mbar_init(B(kKvFull0), 1);
-    mbar_init(B(kKvFull0 + 1), 1);
-    mbar_init(B(kKvEmpty0), 1);
-    mbar_init(B(kKvEmpty0 + 1), 1);
+    for (int i = 0; i < kKStages; ++i) {
+      mbar_init(B(kKFull0 + i), 1);
+      mbar_init(B(kKEmpty0 + i), 1);
+    }
+    for (int i = 0; i < kVStages; ++i) {
+      mbar_init(B(kVFull0 + i), 1);
+      mbar_init(B(kVEmpty0 + i), 1);
+    }
     mbar_init(B(kSFull0), 1);
     mbar_init(B(kSFull0 + 1), 1);
     mbar_init(B(kPFull), 4);
@@ -134,7 +154,43 @@ __global__ void __launch_bounds__(kThreads, 2)
   const uint64_t deadline = globaltimer_ns() + 2000000000ull;
   bool ok = true;
 
-  if (warp == 4) {
+  // Producer of one stream (K by warp 4, V by warp 6): block j's 4 page ids, then its 8 tile copies
+  // into stage j % NS once that stage's previous block has been consumed.
+  auto produce = [&](const CUtensorMap* map, uint32_t off, int ns, int full0, int empty0) {
+    const int oob_row = p.num_blocks * p.num_kv_heads * 16;  // a box starting here is all zero fill
+    for (int j = 0; j < nkb; ++j) {
+      const int st = j % ns;
+      if (j >= ns && !mbar_wait_bounded(B(empty0 + st), ((j / ns) - 1) & 1, deadline)) {
+        atomicOr(p.err, 4u);
+        return;
+      }
+      int ys[kKeys / 16];
+#pragma unroll
+      for (int i = 0; i < kKeys / 16; ++i) {
+        const int page = j * (kKeys / 16) + i;
+        ys[i] = page < npages ? bt[page] : -1;
+      }
+#pragma unroll
+      for (int i = 0; i < kKeys / 16; ++i) {
+        const int page = j * (kKeys / 16) + i;
+        const int bid = ys[i];
+        ys[i] = oob_row;
+        if (page < npages) {
+          if (bid >= 0 && bid < p.num_blocks) ys[i] = (bid * p.num_kv_heads + hk) * 16;
+          else atomicOr(p.err, 1u);
+        }
+      }
+      const uint32_t dst = base + off + st * kTileKV;
+      mbar_arrive_expect_tx(B(full0 + st), kTileKV);
+#pragma unroll
+      for (int i = 0; i < kKeys / 16; ++i)
+        for (int u = 0; u < 2; ++u) tma_load_2d(dst + u * kHalfKV + i * 2048, map, B(full0 + st), u * 64, ys[i]);
+    }
+  };
+
+  if (warp == 6) {
+    if (lane == 0) produce(&vmap, kVOff, kVStages, kVFull0, kVEmpty0);
+  } else if (warp == 4) {
     // ---- producer -------------------------------------------------------------------------------
     if constexpr (kPrefix) {
       if (lane > 0) {
@@ -154,54 +210,20 @@ __global__ void __launch_bounds__(kThreads, 2)
       const int tok0 = q_row0 + tile * (kRows / G);
       tc05::tma_load_3d(base + kQOff, &qmap, B(kQFull), 0, hk * G, tok0);
       tc05::tma_load_3d(base + kQOff + kHalf, &qmap, B(kQFull), 64, hk * G, tok0);
-      const int oob_row = p.num_blocks * p.num_kv_heads * 16;  // a box starting here is all zero fill
-      for (int j = 0; j < nkb && ok; ++j) {
-        const int st = j & 1;
-        if (j >= 2 && !mbar_wait_bounded(B(kKvEmpty0 + st), ((j >> 1) - 1) & 1, deadline)) {
-          ok = false;
-          atomicOr(p.err, 4u);
-          break;
-        }
-        const uint32_t kdst = base + kStageOff + st * 2 * kTileKV, vdst = kdst + kTileKV;
-        // The block's 8 page ids are loaded together, then its 32 tile copies issued.
-        int ys[kKeys / 16];
-#pragma unroll
-        for (int i = 0; i < kKeys / 16; ++i) {
-          const int page = j * (kKeys / 16) + i;
-          ys[i] = page < npages ? bt[page] : -1;
-        }
-#pragma unroll
-        for (int i = 0; i < kKeys / 16; ++i) {
-          const int page = j * (kKeys / 16) + i;
-          const int bid = ys[i];
-          ys[i] = oob_row;
-          if (page < npages) {
-            if (bid >= 0 && bid < p.num_blocks) ys[i] = (bid * p.num_kv_heads + hk) * 16;
-            else atomicOr(p.err, 1u);
-          }
-        }
-        mbar_arrive_expect_tx(B(kKvFull0 + st), 2 * kTileKV);
-#pragma unroll
-        for (int i = 0; i < kKeys / 16; ++i) {
-          const int y = ys[i];
-          for (int u = 0; u < 2; ++u) {
-            tma_load_2d(kdst + u * kHalfKV + i * 2048, &kmap, B(kKvFull0 + st), u * 64, y);
-            tma_load_2d(vdst + u * kHalfKV + i * 2048, &vmap, B(kKvFull0 + st), u * 64, y);
-          }
-        }
-      }
+      produce(&kmap, kKOff, kKStages, kKFull0, kKEmpty0);
     }
   } else if (warp == 5) {
     // ---- MMA issuer ------------------------------------------------------------------------------
     if (lane == 0) {
       constexpr uint32_t idesc_qk = tc05::idesc_f16(kBf16, kRows, kKeys, false, false);
       constexpr uint32_t idesc_pv = tc05::idesc_f16(kBf16, kRows, kD, false, true);
-      // S(j) = Q K(j)^T into S buffer j & 1.
+      // S(j) = Q K(j)^T into S buffer j & 1; K stage j % kKStages is free again once it has run.
       auto issue_qk = [&](int j) -> bool {
-        const int st = j & 1;
-        if (!mbar_wait_bounded(B(kKvFull0 + st), (j >> 1) & 1, deadline)) return false;
+        const int ks_ = j % kKStages;
+        if (!mbar_wait_bounded(B(kKFull0 + ks_), (j / kKStages) & 1, deadline)) return false;
         tc05::fence_after_sync();
-        const uint32_t kbase = base + kStageOff + st * 2 * kTileKV;
+        const uint32_t kbase = base + kKOff + ks_ * kTileKV;
+        const int st = j & 1;
 #pragma unroll
         for (int ks = 0; ks < kD / 16; ++ks) {  // 8 k-steps of 16 along d, 32 bytes apart in a half
           const uint32_t cb = (ks & 3) * 32;
@@ -209,6 +231,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                         tc05::smem_desc_sw128(kbase + (ks >> 2) * kHalfKV + cb, 16, 1024), idesc_qk, ks > 0);
         }
         tc05::commit(B(kSFull0 + st));
+        tc05::commit(B(kKEmpty0 + ks_));
         return true;
       };
       ok = mbar_wait_bounded(B(kQFull), 0, deadline) && issue_qk(0);
@@ -221,22 +244,23 @@ __global__ void __launch_bounds__(kThreads, 2)
             break;
           }
         }
-        if (!mbar_wait_bounded(B(kPFull), j & 1, deadline)) {
+        if (!mbar_wait_bounded(B(kPFull), j & 1, deadline) ||
+            !mbar_wait_bounded(B(kVFull0 + j % kVStages), (j / kVStages) & 1, deadline)) {
           ok = false;
           break;
         }
         tc05::fence_after_sync();
         // O += P V: kKeys / 16 k-steps; P from TMEM (written over S(j), 8 columns = 16 keys per step),
-        // V MN-major in shared memory (16 keys = 2048 B). The next QK into this S buffer is issued
-        // after these MMAs by this thread, and MMAs from one thread execute in order.
-        const uint32_t vbase = base + kStageOff + (j & 1) * 2 * kTileKV + kTileKV;
+        // V MN-major in shared memory (16 keys = 2048 B). The next QK into this S buffer waits until
+        // these MMAs have completed (O_done), since they read P from it.
+        const uint32_t vbase = base + kVOff + (j % kVStages) * kTileKV;
 #pragma unroll
         for (int kt = 0; kt < kKeys / 16; ++kt) {
           tc05::mma_f16_ts(tO, tS0 + (j & 1) * kKeys + kt * 8, tc05::smem_desc_sw128(vbase + kt * 2048, kHalfKV, 1024),
                            idesc_pv, (j > 0 || kt > 0));
         }
         tc05::commit(B(kODone));
-        tc05::commit(B(kKvEmpty0 + (j & 1)));
+        tc05::commit(B(kVEmpty0 + j % kVStages));
       }
       tc05::commit(B(kAllDone));
       mbar_wait_bounded(B(kAllDone), 0, globaltimer_ns() + 1000000000ull);
@@ -329,12 +353,12 @@ __global__ void __launch_bounds__(kThreads, 2)
       tc05::st32u(tS0 + (j & 1) * kKeys + lane_off, w);
       // Keys past every row's limit may hold any bits; zero those V rows so 0 * NaN cannot occur.
       if (t0 + kKeys > max_lim) {
-        const bool landed = mbar_wait_bounded(B(kKvFull0 + (j & 1)), (j >> 1) & 1, deadline);
+        const bool landed = mbar_wait_bounded(B(kVFull0 + j % kVStages), (j / kVStages) & 1, deadline);
         if (!__all_sync(kFull, landed)) {
           ok = false;
           break;
         }
-        const uint32_t vbase = base + kStageOff + (j & 1) * 2 * kTileKV + kTileKV;
+        const uint32_t vbase = base + kVOff + (j % kVStages) * kTileKV;
         const int first = max_lim - t0;  // rows [first, kKeys) of the V tile, both halves
         for (int idx = r; idx < (kKeys - first) * 16; idx += 128) {
           const int row = first + idx / 16, c16 = idx % 16;
@@ -351,7 +375,9 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     // Epilogue: O / l -> out rows, or (prefix) the row's (m, l, O) -> its workspace slot.
     if (ok) {
-      const bool done = __all_sync(kFull, mbar_wait_bounded(B(kODone), (nkb - 1) & 1, deadline));
+      // All MMAs done: the issuer's final commit. (A parity wait on O_done for the last block could
+      // return early while the previous P.V is still pending, since O_done may then be two phases back.)
+      const bool done = __all_sync(kFull, mbar_wait_bounded(B(kAllDone), 0, deadline));
       if (done) tc05::fence_after_sync();
       if (!done) {
         ok = false;

@@ -100,6 +100,23 @@ def test_tcgen05_and_warp_mma_prefill_agree():
     assert (outs[0].double() - outs[1].double()).abs().max().item() <= 2 * TOL["bf16"]
 
 
+def test_tcgen05_prefill_is_deterministic():
+    """Repeated launches give bit-identical outputs: a pipeline race (a buffer reused before the MMA
+    reading it finished) shows up as run-to-run differences, even where it stays within tolerance."""
+    ctxs, news, hq, hkv, d = [2000, 1500, 333], [2000, 700, 333], 32, 8, 128
+    bt, kc, vc, q, qs = _build(ctxs, news, hq, hkv, d, torch.bfloat16, seed=41)
+    lens = torch.tensor(ctxs, dtype=torch.int32).cuda()
+    outs = []
+    for _ in range(6):
+        out = torch.empty(q.shape[0], hq, d, dtype=torch.bfloat16, device="cuda")
+        pa.pa_prefill(out, q.cuda(), kc, vc, bt.cuda(), qs.cuda(), lens, max(news), d ** -0.5, hkv, kernel=1)
+        outs.append(out)
+    torch.cuda.synchronize()
+    assert pa.pa_read_device_error(clear=True) == 0
+    for o in outs[1:]:
+        assert torch.equal(o.view(torch.int16), outs[0].view(torch.int16))
+
+
 def test_chunked_equals_whole_and_last_row_equals_decode():
     ctxs, hq, hkv, d = [100], 8, 2, 128
     bt, kc, vc, q, _ = _build(ctxs, [100], hq, hkv, d, torch.bfloat16, seed=5)
