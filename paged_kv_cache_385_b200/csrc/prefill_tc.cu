@@ -17,8 +17,9 @@
 //                               max / sum in registers, P (bf16/f16) written back to TMEM over S,
 //                               O rescaled in TMEM only when a row's max grew past the lazy bound
 //   O[128 x 128] += P . V       A = P from TMEM, B = V (MN-major: d contiguous), D in TMEM
-// Warps: 0-3 softmax + epilogue, 4 TMA producer of Q and K (3-stage ring), 5 MMA issuer (one
-// thread) and TMEM owner, 6 TMA producer of V (2-stage ring). Every mbarrier wait is bounded.
+// Warps: 0-3 softmax + epilogue, 4 TMA producer of Q and K (3-stage ring), 5 QK issuer (one thread)
+// and TMEM owner, 6 TMA producer of V (2-stage ring), 7 PV issuer (one thread). Every mbarrier wait
+// is bounded.
 #include "internal.h"
 #include "pa_device.cuh"
 #include "tc05.cuh"
@@ -28,7 +29,7 @@ namespace {
 
 constexpr int kD = 128;
 constexpr int kRows = 128;   // query rows per CTA
-constexpr int kThreads = 224;
+constexpr int kThreads = 256;
 constexpr uint32_t kHalf = 16384;  // one 64-element (128-byte) column half of a 128-row tile
 constexpr uint32_t kTile = 2 * kHalf;
 
@@ -213,14 +214,19 @@ __global__ void __launch_bounds__(kThreads, 2)
       produce(&kmap, kKOff, kKStages, kKFull0, kKEmpty0);
     }
   } else if (warp == 5) {
-    // ---- MMA issuer ------------------------------------------------------------------------------
+    // ---- QK issuer: S(j) = Q K(j)^T into S buffer j & 1 ------------------------------------------
     if (lane == 0) {
       constexpr uint32_t idesc_qk = tc05::idesc_f16(kBf16, kRows, kKeys, false, false);
-      constexpr uint32_t idesc_pv = tc05::idesc_f16(kBf16, kRows, kD, false, true);
-      // S(j) = Q K(j)^T into S buffer j & 1; K stage j % kKStages is free again once it has run.
-      auto issue_qk = [&](int j) -> bool {
+      ok = mbar_wait_bounded(B(kQFull), 0, deadline);
+      for (int j = 0; j < nkb && ok; ++j) {
+        // Buffer j & 1 holds P(j-2) until P(j-2).V has completed. O_done's phases are waited in
+        // order (j - 2 = 0, 1, ...), so this parity wait cannot be taken for an older phase.
         const int ks_ = j % kKStages;
-        if (!mbar_wait_bounded(B(kKFull0 + ks_), (j / kKStages) & 1, deadline)) return false;
+        if ((j >= 2 && !mbar_wait_bounded(B(kODone), (j - 2) & 1, deadline)) ||
+            !mbar_wait_bounded(B(kKFull0 + ks_), (j / kKStages) & 1, deadline)) {
+          ok = false;
+          break;
+        }
         tc05::fence_after_sync();
         const uint32_t kbase = base + kKOff + ks_ * kTileKV;
         const int st = j & 1;
@@ -231,28 +237,25 @@ __global__ void __launch_bounds__(kThreads, 2)
                         tc05::smem_desc_sw128(kbase + (ks >> 2) * kHalfKV + cb, 16, 1024), idesc_qk, ks > 0);
         }
         tc05::commit(B(kSFull0 + st));
-        tc05::commit(B(kKEmpty0 + ks_));
-        return true;
-      };
-      ok = mbar_wait_bounded(B(kQFull), 0, deadline) && issue_qk(0);
+        tc05::commit(B(kKEmpty0 + ks_));  // K stage free again once this QK has run
+      }
+      if (!ok) atomicOr(p.err, 4u);
+    }
+  } else if (warp == 7) {
+    // ---- PV issuer: O += P(j) V(j) ------------------------------------------------------------------
+    // A separate thread from the QK issuer, so that P(j).V is issued as soon as P(j) is ready even
+    // while the QK issue of a later block waits for room in the tensor pipe.
+    if (lane == 0) {
+      constexpr uint32_t idesc_pv = tc05::idesc_f16(kBf16, kRows, kD, false, true);
       for (int j = 0; j < nkb && ok; ++j) {
-        // S(j+1) goes to the buffer that holds P(j-1): softmax(j-1) is done with it (p_full(j-1) was
-        // seen), but P(j-1) . V may still be reading it, so wait for that MMA to finish first.
-        if (j + 1 < nkb) {
-          if ((j > 0 && !mbar_wait_bounded(B(kODone), (j - 1) & 1, deadline)) || !issue_qk(j + 1)) {
-            ok = false;
-            break;
-          }
-        }
         if (!mbar_wait_bounded(B(kPFull), j & 1, deadline) ||
             !mbar_wait_bounded(B(kVFull0 + j % kVStages), (j / kVStages) & 1, deadline)) {
           ok = false;
           break;
         }
         tc05::fence_after_sync();
-        // O += P V: kKeys / 16 k-steps; P from TMEM (written over S(j), 8 columns = 16 keys per step),
-        // V MN-major in shared memory (16 keys = 2048 B). The next QK into this S buffer waits until
-        // these MMAs have completed (O_done), since they read P from it.
+        // kKeys / 16 k-steps; P from TMEM (written over S(j), 8 columns = 16 keys per step), V
+        // MN-major in shared memory (16 keys = 2048 B).
         const uint32_t vbase = base + kVOff + (j % kVStages) * kTileKV;
 #pragma unroll
         for (int kt = 0; kt < kKeys / 16; ++kt) {
@@ -262,6 +265,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         tc05::commit(B(kODone));
         tc05::commit(B(kVEmpty0 + j % kVStages));
       }
+      // Every QK has completed before its softmax finished, so this covers all of the CTA's MMAs.
       tc05::commit(B(kAllDone));
       mbar_wait_bounded(B(kAllDone), 0, globaltimer_ns() + 1000000000ull);
       if (!ok) atomicOr(p.err, 4u);
