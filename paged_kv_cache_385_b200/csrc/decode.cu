@@ -480,6 +480,10 @@ __global__ void __launch_bounds__(Cfg<KV, QT, D, NT, KIND, OCC>::kThreads, Cfg<K
   const int Hq = p.num_kv_heads * G;
   const int PT = p.partition_tokens;
 
+  // The block-table entry of this lane's page, read before the context length is known so that the
+  // two loads overlap (entries past the context are masked below; the read stays inside the table).
+  const int j_lane = p.start_tokens / 16 + part * (PT / 16) + warp + lane * C::kWarps;
+  const int bid_lane = j_lane < p.max_blocks ? p.block_tables[s * p.bt_stride + j_lane] : -1;
   // This grid covers tokens [start, start + span) of the sequence: all of it for plain decode, the
   // part after the shared prefix for cascade decode.
   const int ctx = p.context_lens[s];
@@ -579,8 +583,7 @@ __global__ void __launch_bounds__(Cfg<KV, QT, D, NT, KIND, OCC>::kThreads, Cfg<K
   const int n_w = max(0, (j1 - j0 - warp + C::kWarps - 1) / C::kWarps);  // pages of this warp (<= 32)
 
   // Physical block of this warp's i-th page sits in lane i.
-  int my_bid = -1;
-  if (lane < n_w) my_bid = p.block_tables[s * p.bt_stride + j0 + warp + lane * C::kWarps];
+  const int my_bid = lane < n_w ? bid_lane : -1;
   const bool my_bad = lane < n_w && (my_bid < 0 || my_bid >= p.num_blocks);
   if (__any_sync(kFull, my_bad) && lane == 0) atomicOr(p.err, 1u);
 
@@ -702,49 +705,86 @@ __global__ void __launch_bounds__(Cfg<KV, QT, D, NT, KIND, OCC>::kThreads, Cfg<K
 
   const bool inline_merge = p.merge_prefix_inline && nparts <= 1;
   const bool direct = (!p.always_partials && nparts <= 1) || inline_merge;
-  for (int idx = threadIdx.x; idx < G * D; idx += C::kThreads) {
-    const int g = idx / D, d = idx % D;
-    float M = -INFINITY;
+  // Each thread owns one d and four group members at a time (g = gb .. gb + 3; members past G are
+  // computed on a clamped g and dropped).
+  static_assert(C::kThreads % D == 0, "threads must cover whole rows of d");
+  constexpr int kDPar = C::kThreads / D;
+  const int d = threadIdx.x % D;
+  const int npre = p.part_offset;
+  for (int gb = (threadIdx.x / D) * 4; gb < G; gb += kDPar * 4) {
+    float M[4], num[4], den[4];
 #pragma unroll
-    for (int w = 0; w < C::kWarps; ++w) M = fmaxf(M, mg[w * C::kGPad + g]);
-    float num = 0.f, den = 0.f;
+    for (int u = 0; u < 4; ++u) {
+      const int g = min(gb + u, G - 1);
+      M[u] = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < C::kWarps; ++w) {
-      const float f = ex2(mg[w * C::kGPad + g] - M);
-      num = fmaf(f, ag[(w * C::kGPad + g) * D + d], num);
-      den = fmaf(f, lg[w * C::kGPad + g], den);
+      for (int w = 0; w < C::kWarps; ++w) M[u] = fmaxf(M[u], mg[w * C::kGPad + g]);
+      num[u] = 0.f;
+      den[u] = 0.f;
+#pragma unroll
+      for (int w = 0; w < C::kWarps; ++w) {
+        const float f = ex2(mg[w * C::kGPad + g] - M[u]);
+        num[u] = fmaf(f, ag[(w * C::kGPad + g) * D + d], num[u]);
+        den[u] = fmaf(f, lg[w * C::kGPad + g], den[u]);
+      }
     }
-    const int h = hk * G + g;
     if (inline_merge) {
-      // Fold in the shared-prefix partials (slots 0 .. part_offset - 1), prefix first, then this CTA.
-      const int64_t row0 = (static_cast<int64_t>(s) * Hq + h) * p.ws_parts;
-      float Mp = M;
-      for (int k = 0; k < p.part_offset; ++k) Mp = fmaxf(Mp, p.ws_ml[(row0 + k) * 2]);
-      float n2 = 0.f, d2 = 0.f;
-      for (int k = 0; k < p.part_offset; ++k) {
-        const float f = ex2(p.ws_ml[(row0 + k) * 2] - Mp);
-        n2 = fmaf(f, p.ws_acc[(row0 + k) * D + d], n2);
-        d2 = fmaf(f, p.ws_ml[(row0 + k) * 2 + 1], d2);
+      // Fold in the shared-prefix partials (workspace slots 0 .. npre - 1), four slots of four members
+      // per round: every load of a round is issued before any of them is used.
+      for (int k0 = 0; k0 < npre; k0 += 4) {
+        float pm[4][4], pl[4][4], pa[4][4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int64_t row0 = (static_cast<int64_t>(s) * Hq + hk * G + min(gb + u, G - 1)) * p.ws_parts;
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            const int64_t slot = row0 + min(k0 + v, npre - 1);
+            const float2 ml = *reinterpret_cast<const float2*>(p.ws_ml + slot * 2);
+            pm[u][v] = k0 + v < npre ? ml.x : -INFINITY;
+            pl[u][v] = ml.y;
+            pa[u][v] = p.ws_acc[slot * D + d];
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          float Mn = M[u];
+#pragma unroll
+          for (int v = 0; v < 4; ++v) Mn = fmaxf(Mn, pm[u][v]);
+          if (Mn == -INFINITY) continue;
+          const float a = ex2(M[u] - Mn);
+          num[u] *= a;
+          den[u] *= a;
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            const float f = ex2(pm[u][v] - Mn);
+            num[u] = fmaf(f, pa[u][v], num[u]);
+            den[u] = fmaf(f, pl[u][v], den[u]);
+          }
+          M[u] = Mn;
+        }
       }
-      const float f = ex2(M - Mp);
-      num = fmaf(f, num, n2);
-      den = fmaf(f, den, d2);
     }
-    if (direct) {
-      const float o = num / den * p.v_scale;
-      out_t bits;
-      if constexpr (C::kQBf16) {
-        bits = __bfloat16_as_ushort(__float2bfloat16_rn(o));
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int g = gb + u;
+      if (g >= G) break;
+      const int h = hk * G + g;
+      if (direct) {
+        const float o = num[u] / den[u] * p.v_scale;
+        out_t bits;
+        if constexpr (C::kQBf16) {
+          bits = __bfloat16_as_ushort(__float2bfloat16_rn(o));
+        } else {
+          bits = __half_as_ushort(__float2half_rn(o));
+        }
+        static_cast<out_t*>(p.out)[s * p.o_stride_s + h * p.o_stride_h + d] = bits;
       } else {
-        bits = __half_as_ushort(__float2half_rn(o));
-      }
-      static_cast<out_t*>(p.out)[s * p.o_stride_s + h * p.o_stride_h + d] = bits;
-    } else {
-      const int64_t row = (static_cast<int64_t>(s) * Hq + h) * p.ws_parts + p.part_offset + part;
-      p.ws_acc[row * D + d] = num;
-      if (d == 0) {
-        p.ws_ml[row * 2] = M;
-        p.ws_ml[row * 2 + 1] = den;
+        const int64_t row = (static_cast<int64_t>(s) * Hq + h) * p.ws_parts + p.part_offset + part;
+        p.ws_acc[row * D + d] = num[u];
+        if (d == 0) {
+          p.ws_ml[row * 2] = M[u];
+          p.ws_ml[row * 2 + 1] = den[u];
+        }
       }
     }
   }
