@@ -484,6 +484,29 @@ __global__ void __launch_bounds__(Cfg<KV, QT, D, NT, KIND, OCC>::kThreads, Cfg<K
   // two loads overlap (entries past the context are masked below; the read stays inside the table).
   const int j_lane = p.start_tokens / 16 + part * (PT / 16) + warp + lane * C::kWarps;
   const int bid_lane = j_lane < p.max_blocks ? p.block_tables[s * p.bt_stride + j_lane] : -1;
+  // Cascade: the CTA of KV head 0, partition 0 of each sequence checks that its table maps the
+  // shared prefix pages to sequence 0's blocks (the prefix kernels read sequence 0's). The first
+  // 2 * kThreads entries are read here and compared later, so the reads overlap the page loop.
+  const bool chk = p.start_tokens > 0 && hk == 0 && part == 0;
+  const int npre_pages = p.start_tokens / 16;
+  int chk_a[2] = {0, 0}, chk_b[2] = {0, 0};
+  if (chk) {
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int j = threadIdx.x + u * C::kThreads;
+      if (j < npre_pages) {
+        chk_a[u] = p.block_tables[s * p.bt_stride + j];
+        chk_b[u] = p.block_tables[j];
+      }
+    }
+  }
+  auto prefix_check = [&]() {
+    if (!chk) return;
+    bool bad = chk_a[0] != chk_b[0] || chk_a[1] != chk_b[1];
+    for (int j = threadIdx.x + 2 * C::kThreads; j < npre_pages; j += C::kThreads)
+      bad |= p.block_tables[s * p.bt_stride + j] != p.block_tables[j];
+    if (bad) atomicOr(p.err, 16u);
+  };
   // This grid covers tokens [start, start + span) of the sequence: all of it for plain decode, the
   // part after the shared prefix for cascade decode.
   const int ctx = p.context_lens[s];
@@ -540,6 +563,7 @@ __global__ void __launch_bounds__(Cfg<KV, QT, D, NT, KIND, OCC>::kThreads, Cfg<K
   }
 
   typedef uint16_t out_t;
+  if (span == 0) prefix_check();
   if (span == 0 && late_wait) pdl_wait();
   if (span == 0 && p.merge_prefix_inline) {
     // Nothing past the shared prefix: the output is the merge of the prefix partials alone.
@@ -684,6 +708,7 @@ __global__ void __launch_bounds__(Cfg<KV, QT, D, NT, KIND, OCC>::kThreads, Cfg<K
     if (lane == 0) atomicOr(p.err, 4u);
   }
   const int any_fail = __syncthreads_or(!ok);
+  prefix_check();
   pdl_launch_dependents();
   if (late_wait) pdl_wait();  // the prefix partials (and the prefix grid's completion) from here on
 
@@ -735,14 +760,15 @@ __global__ void __launch_bounds__(Cfg<KV, QT, D, NT, KIND, OCC>::kThreads, Cfg<K
         float pm[4][4], pl[4][4], pa[4][4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          const int64_t row0 = (static_cast<int64_t>(s) * Hq + hk * G + min(gb + u, G - 1)) * p.ws_parts;
+          const int g = min(gb + u, G - 1);
+          const int64_t row0 = (static_cast<int64_t>(s) * Hq + hk * G + g) * p.ws_parts;
 #pragma unroll
           for (int v = 0; v < 4; ++v) {
-            const int64_t slot = row0 + min(k0 + v, npre - 1);
-            const float2 ml = *reinterpret_cast<const float2*>(p.ws_ml + slot * 2);
+            const int k = min(k0 + v, npre - 1);
+            const float2 ml = *reinterpret_cast<const float2*>(p.ws_ml + (row0 + k) * 2);
+            pa[u][v] = p.ws_acc[(row0 + k) * D + d];
             pm[u][v] = k0 + v < npre ? ml.x : -INFINITY;
             pl[u][v] = ml.y;
-            pa[u][v] = p.ws_acc[slot * D + d];
           }
         }
 #pragma unroll

@@ -160,17 +160,6 @@ __global__ void __launch_bounds__(PCfg<KV, D>::kThreads) mq_kernel(const __grid_
   int lim_max = max(lim_lo, lim_hi);
   for (int off = 4; off < 32; off <<= 1) lim_max = max(lim_max, __shfl_xor_sync(kFull, lim_max, off));
 
-  if constexpr (!kPrefill) {
-    // Every sequence of these rows must map the prefix pages of this chunk to sequence 0's blocks.
-    const int s_first = min(tile * kRowsPerCta + warp * 16, num_rows - 1) / G;
-    const int s_last = min(tile * kRowsPerCta + warp * 16 + 15, num_rows - 1) / G;
-    bool mismatch = false;
-    for (int idx = lane; idx < (s_last - s_first + 1) * npages; idx += 32) {
-      const int sq = s_first + idx / npages, j = j0 + idx % npages;
-      mismatch |= p.block_tables[sq * p.bt_stride + j] != p.block_tables[j];
-    }
-    if (__any_sync(kFull, mismatch) && lane == 0) atomicOr(p.err, 16u);
-  }
 
   uint32_t qa[KS][4];
   {

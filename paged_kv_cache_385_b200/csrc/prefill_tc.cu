@@ -193,18 +193,6 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (lane == 0) produce(&vmap, kVOff, kVStages, kVFull0, kVEmpty0);
   } else if (warp == 4) {
     // ---- producer -------------------------------------------------------------------------------
-    if constexpr (kPrefix) {
-      if (lane > 0) {
-        // Lanes 1-31: every sequence of the tile must map this chunk's pages to sequence 0's blocks.
-        const int s0 = tile * kRows / G, s1 = min((tile + 1) * kRows, num_rows) / G;  // [s0, s1)
-        bool mismatch = false;
-        for (int idx = lane - 1; idx < (s1 - s0) * npages; idx += 31) {
-          const int sq = s0 + idx / npages, i = idx % npages;
-          mismatch |= p.block_tables[static_cast<int64_t>(sq) * p.bt_stride + key0 / 16 + i] != bt[i];
-        }
-        if (mismatch) atomicOr(p.err, 16u);
-      }
-    }
     if (lane == 0) {
       prefetch_tensormap(&qmap);
       mbar_arrive_expect_tx(B(kQFull), kTile);
@@ -386,20 +374,35 @@ __global__ void __launch_bounds__(kThreads, 2)
       if (!done) {
         ok = false;
       } else if constexpr (kPrefix) {
-        const int Hq = p.num_kv_heads * G;
-        const int64_t slot = (static_cast<int64_t>(valid ? R / G : 0) * Hq + hk * G + R % G) * p.ws_parts + s;
-        float* dst = p.ws_acc + slot * kD;
+        // O rows go through shared memory (the K/V stages are idle now) and leave it as one bulk
+        // copy per 512-byte workspace row. (That every sequence maps the prefix pages to sequence 0's
+        // blocks is checked by the suffix decode, off this kernel's critical path.)
+        constexpr uint32_t kRowStride = (kD + 4) * 4;  // padded: row-wise writes free of bank conflicts
+        const uint32_t stg = base + kKOff + warp * 32 * kRowStride;
+        static_assert(kKOff + 4 * 32 * kRowStride <= kBarOff, "staging fits the K/V stages");
 #pragma unroll
         for (int c = 0; c < kD / 32; ++c) {
           float v[32];
           tc05::ld32(tO + lane_off + c * 32, v);
-          if (valid) {
 #pragma unroll
-            for (int q = 0; q < 8; ++q)
-              *reinterpret_cast<float4*>(dst + c * 32 + 4 * q) = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-          }
+          for (int q = 0; q < 8; ++q)
+            asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(stg + lane * kRowStride + (c * 32 + 4 * q) * 4),
+                         "f"(v[4 * q]), "f"(v[4 * q + 1]), "f"(v[4 * q + 2]), "f"(v[4 * q + 3])
+                         : "memory");
         }
-        if (valid) *reinterpret_cast<float2*>(p.ws_ml + slot * 2) = make_float2(m, l);
+        // Each valid row's lane issues the bulk copy of its own staged row (512 bytes, 16-byte
+        // aligned at both ends), after a proxy fence makes its shared-memory writes visible to it.
+        const int Hq = p.num_kv_heads * G;
+        if (valid) {
+          const int64_t slot = (static_cast<int64_t>(R / G) * Hq + hk * G + R % G) * p.ws_parts + s;
+          *reinterpret_cast<float2*>(p.ws_ml + slot * 2) = make_float2(m, l);
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(p.ws_acc + slot * kD),
+                       "r"(stg + lane * kRowStride), "r"(kD * 4)
+                       : "memory");
+          asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+          asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");  // before the CTA's smem goes
+        }
       } else {
         const float inv = l > 0.f ? 1.f / l : 0.f;
         uint16_t* dst = static_cast<uint16_t*>(p.out) + static_cast<int64_t>(q_row0 + (valid ? R / G : 0)) * p.o_stride_t +
