@@ -816,10 +816,17 @@ __global__ void __launch_bounds__(Cfg<KV, QT, D, NT, KIND, OCC>::kThreads, Cfg<K
   }
 }
 
-// Merge the partitions of each (sequence, query head) in index order.
+// Merge the partitions of each (sequence, query head). blockDim.x / D groups (1 .. kReduceSplit) of D
+// threads take partitions k = w, w + groups, ... (eight per round, all of a round's loads in flight),
+// each keeping a running (M, num, den); the groups are then combined in fixed order, so the result is
+// deterministic. Many partitions get several groups; a handful get one.
+constexpr int kReduceSplit = 4;
 template <int D, bool kBf16>
-__global__ void __launch_bounds__(D) reduce_kernel(const DecodeParams p) {
-  const int h = blockIdx.x, s = blockIdx.y, d = threadIdx.x;
+__global__ void __launch_bounds__(kReduceSplit * D) reduce_kernel(const DecodeParams p) {
+  const int h = blockIdx.x, s = blockIdx.y, d = threadIdx.x % D, w = threadIdx.x / D;
+  const int groups = blockDim.x / D;
+  __shared__ float sm_num[kReduceSplit][D];
+  __shared__ float sm_m[kReduceSplit], sm_den[kReduceSplit];
   pdl_wait();  // the partials come from the decode grid just before this one
   pdl_launch_dependents();
   const int Hq = p.num_kv_heads * p.group;
@@ -829,25 +836,56 @@ __global__ void __launch_bounds__(D) reduce_kernel(const DecodeParams p) {
   const int np = p.part_offset + (span + PT - 1) / PT;
   if (!p.always_partials && np <= 1) return;  // the decode kernel wrote this row
   const int64_t row0 = (static_cast<int64_t>(s) * Hq + h) * p.ws_parts;
-  float M = -INFINITY;
-  for (int k = 0; k < np; ++k) M = fmaxf(M, p.ws_ml[(row0 + k) * 2]);
-  if (M == -INFINITY) {  // no token at all (empty context)
-    static_cast<uint16_t*>(p.out)[s * p.o_stride_s + h * p.o_stride_h + d] = 0;
-    return;
+  float M = -INFINITY, num = 0.f, den = 0.f;
+  for (int k0 = w; k0 < np; k0 += 8 * groups) {
+    float mk[8], lk[8], ak[8];
+#pragma unroll
+    for (int v = 0; v < 8; ++v) {
+      const int k = k0 + v * groups;
+      const int64_t slot = row0 + min(k, np - 1);
+      const float2 ml = *reinterpret_cast<const float2*>(p.ws_ml + slot * 2);
+      mk[v] = k < np ? ml.x : -INFINITY;
+      lk[v] = ml.y;
+      ak[v] = p.ws_acc[slot * D + d];
+    }
+    float Mn = M;
+#pragma unroll
+    for (int v = 0; v < 8; ++v) Mn = fmaxf(Mn, mk[v]);
+    if (Mn == -INFINITY) continue;
+    const float a = ex2(M - Mn);
+    num *= a;
+    den *= a;
+#pragma unroll
+    for (int v = 0; v < 8; ++v) {
+      const float f = ex2(mk[v] - Mn);
+      num = fmaf(f, ak[v], num);
+      den = fmaf(f, lk[v], den);
+    }
+    M = Mn;
   }
-  float num = 0.f, den = 0.f;
-#pragma unroll 4
-  for (int k = 0; k < np; ++k) {
-    const float f = ex2(p.ws_ml[(row0 + k) * 2] - M);
-    num = fmaf(f, p.ws_acc[(row0 + k) * D + d], num);
-    den = fmaf(f, p.ws_ml[(row0 + k) * 2 + 1], den);
+  sm_num[w][d] = num;
+  if (d == 0) {
+    sm_m[w] = M;
+    sm_den[w] = den;
   }
-  const float o = num / den * p.v_scale;
-  uint16_t bits;
-  if constexpr (kBf16) {
-    bits = __bfloat16_as_ushort(__float2bfloat16_rn(o));
-  } else {
-    bits = __half_as_ushort(__float2half_rn(o));
+  __syncthreads();
+  if (w != 0) return;
+  float Mt = -INFINITY;
+  for (int g = 0; g < groups; ++g) Mt = fmaxf(Mt, sm_m[g]);
+  uint16_t bits = 0;  // no token at all (empty context): 0
+  if (Mt != -INFINITY) {
+    float nt = 0.f, dt = 0.f;
+    for (int g = 0; g < groups; ++g) {
+      const float f = ex2(sm_m[g] - Mt);  // a group without partitions has m = -inf: weight 0
+      nt = fmaf(f, sm_num[g][d], nt);
+      dt = fmaf(f, sm_den[g], dt);
+    }
+    const float o = nt / dt * p.v_scale;
+    if constexpr (kBf16) {
+      bits = __bfloat16_as_ushort(__float2bfloat16_rn(o));
+    } else {
+      bits = __half_as_ushort(__float2half_rn(o));
+    }
   }
   static_cast<uint16_t*>(p.out)[s * p.o_stride_s + h * p.o_stride_h + d] = bits;
 }
@@ -942,11 +980,12 @@ cudaError_t launch_decode(const DecodeConfig& c, const CUtensorMap& km, const CU
 cudaError_t launch_reduce(const DecodeConfig& c, const DecodeParams& p, cudaStream_t st) {
   const dim3 grid(p.num_kv_heads * p.group, p.num_seqs);
   const bool bf = c.q == QType::BF16;
+  const unsigned groups = p.ws_parts > 8 ? kReduceSplit : 1;
   if (c.head_dim == 128)
-    return bf ? launch_pdl(reduce_kernel<128, true>, grid, dim3(128), 0, st, p)
-              : launch_pdl(reduce_kernel<128, false>, grid, dim3(128), 0, st, p);
-  return bf ? launch_pdl(reduce_kernel<64, true>, grid, dim3(64), 0, st, p)
-            : launch_pdl(reduce_kernel<64, false>, grid, dim3(64), 0, st, p);
+    return bf ? launch_pdl(reduce_kernel<128, true>, grid, dim3(groups * 128), 0, st, p)
+              : launch_pdl(reduce_kernel<128, false>, grid, dim3(groups * 128), 0, st, p);
+  return bf ? launch_pdl(reduce_kernel<64, true>, grid, dim3(groups * 64), 0, st, p)
+            : launch_pdl(reduce_kernel<64, false>, grid, dim3(groups * 64), 0, st, p);
 }
 
 uint32_t* decode_error_word() {
