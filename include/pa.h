@@ -185,6 +185,7 @@ int pa_copy_blocks(pa_tensor* k_cache, pa_tensor* v_cache, const pa_tensor* bloc
  *                 and read-only here: copy-on-write them first), else it is skipped with
  *                 PA_DEVERR_BAD_SLOT.
  *   F16/BF16 caches only. A workspace is always needed: pa_decode_cascade_workspace_bytes.
+ *   opts->prefix_kernel picks the kernel of the shared part (tcgen05 by default where it applies).
  *   A block table that does not share the prefix blocks sets PA_DEVERR_PREFIX (results undefined;
  *   every row's first shared_prefix_tokens / 16 entries are compared with row 0's).
  * Source: "vLLM 前世今生" section 3.2 (sequences pointing at the same physical blocks; prefix
