@@ -645,6 +645,11 @@ int pa_prefill(pa_tensor* out, const pa_tensor* q, const pa_tensor* k_cache, con
   if (!out->data || !q->data || !k_cache->data || !v_cache->data || !block_tables->data || !query_start->data ||
       !context_lens->data)
     return fail(PA_ERR_INVALID_ARG, "NULL data pointer");
+  // The kernel choice is an argument error, reported before any device call.
+  const int G = static_cast<int>(Hq / num_kv_heads);
+  if (kernel < -1 || kernel > 1) return fail(PA_ERR_INVALID_ARG, "kernel must be -1, 0 or 1");
+  const bool tc_ok = pa::prefill_tc_supported(static_cast<int>(D), G);
+  if (kernel == 1 && !tc_ok) return fail(PA_ERR_UNSUPPORTED, "the tcgen05 prefill needs head_dim 128 and a group dividing 128");
   pa::MqParams p{};
   p.q = q->data;
   p.q_stride_s = q->stride[0];
@@ -667,10 +672,6 @@ int pa_prefill(pa_tensor* out, const pa_tensor* q, const pa_tensor* k_cache, con
   CUtensorMap km, vm;
   if ((st = encode_pool_map(&km, k_cache, 2)) || (st = encode_pool_map(&vm, v_cache, 2))) return st;
   const pa::KvType kv = cd == PA_BF16 ? pa::KvType::BF16 : pa::KvType::F16;
-  const int G = static_cast<int>(Hq / num_kv_heads);
-  if (kernel < -1 || kernel > 1) return fail(PA_ERR_INVALID_ARG, "kernel must be -1, 0 or 1");
-  const bool tc_ok = pa::prefill_tc_supported(static_cast<int>(D), G);
-  if (kernel == 1 && !tc_ok) return fail(PA_ERR_UNSUPPORTED, "the tcgen05 prefill needs head_dim 128 and a group dividing 128");
   cudaError_t e;
   if (kernel == 1 || (kernel == -1 && tc_ok)) {
     CUtensorMap qm;

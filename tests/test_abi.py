@@ -145,3 +145,56 @@ def test_slot_helper_rejects_out_of_range():
     with pytest.raises(pa.PagedAttentionError):
         pa.pa_slots_for_positions(bt, [0], [40])  # beyond the table
     assert pa.pa_slots_for_positions(bt, [0], [5]).tolist() == [53]
+
+
+def _aligned_zeros(shape, dtype, align=256):
+    """A zeroed host tensor whose data starts on an `align`-byte boundary (the library checks it)."""
+    n = int(np.prod(shape)) * torch.tensor([], dtype=dtype).element_size()
+    raw = torch.zeros(n + align, dtype=torch.uint8)
+    off = (-raw.data_ptr()) % align
+    return raw[off:off + n].view(dtype).view(*shape)
+
+
+def test_cascade_option_validation_happens_on_the_host():
+    """A bad opts.prefix_kernel or an unaligned prefix length is refused before any device work (the
+    tensors here are host memory, which no kernel could read)."""
+    B, Hq, Hkv, D, NB = 2, 8, 2, 128, 16
+    q = _aligned_zeros((B, Hq, D), torch.bfloat16)
+    kc = _aligned_zeros((NB, Hkv, 16, D), torch.bfloat16)
+    bt = torch.zeros(B, 4, dtype=torch.int32)
+    lens = torch.full((B,), 40, dtype=torch.int32)
+    ts = [pa.as_pa_tensor(t, n, device=False) for t, n in ((q, "out"), (q, "q"), (kc, "k"), (kc, "v"), (bt, "bt"),
+                                                            (lens, "lens"))]
+    lib = pa.lib()
+
+    def call(prefix_tokens, **kw):
+        opts = pa.PaDecodeOpts()
+        lib.pa_decode_opts_init(ctypes.byref(opts))
+        for k, v in kw.items():
+            setattr(opts, k, v)
+        out, qq, k, v, b, n = [ctypes.byref(t) for t in ts]
+        return lib.pa_decode_cascade(out, qq, None, None, None, k, v, b, n, prefix_tokens, 0.088, Hkv,
+                                     ctypes.byref(opts), None)
+
+    assert call(32, prefix_kernel=7) == pa.PA_ERR_INVALID_ARG
+    assert "prefix_kernel" in pa.pa_last_error()
+    assert call(24) == pa.PA_ERR_INVALID_ARG  # not a multiple of 16
+    assert "multiple of 16" in pa.pa_last_error()
+
+
+def test_prefill_kernel_choice_is_checked_on_the_host():
+    """The tcgen05 prefill takes head_dim 128 and a group dividing 128: asking for it with D = 64 is
+    refused before any device work; an unknown kernel number too."""
+    T, Hq, Hkv, D, NB, B = 8, 4, 4, 64, 4, 1
+    q = _aligned_zeros((T, Hq, D), torch.float16)
+    kc = _aligned_zeros((NB, Hkv, 16, D), torch.float16)
+    bt = torch.zeros(B, 1, dtype=torch.int32)
+    qs = torch.tensor([0, T], dtype=torch.int32)
+    lens = torch.tensor([T], dtype=torch.int32)
+    ts = [pa.as_pa_tensor(t, n, device=False) for t, n in ((q, "out"), (q, "q"), (kc, "k"), (kc, "v"), (bt, "bt"),
+                                                            (qs, "qs"), (lens, "lens"))]
+    lib = pa.lib()
+    args = [ctypes.byref(t) for t in ts]
+    assert lib.pa_prefill(*args, T, 0.125, Hkv, 1, None) == pa.PA_ERR_UNSUPPORTED
+    assert "tcgen05" in pa.pa_last_error()
+    assert lib.pa_prefill(*args, T, 0.125, Hkv, 5, None) == pa.PA_ERR_INVALID_ARG
