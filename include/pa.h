@@ -276,6 +276,14 @@ int pa_read_device_error(uint32_t* bits, int clear);
 /* Library version, "major.minor.patch". */
 const char* pa_version(void);
 
+/* Self-test of the bounded waits every kernel uses on its asynchronous-copy and MMA barriers (no
+ * counterpart on the pages): launches one CTA on `stream` that waits on a barrier nothing ever
+ * arrives on, gives up after timeout_us microseconds (1 .. 1000000) of global time, and ORs
+ * PA_DEVERR_TIMEOUT into error_word (a device int32; NULL = the library's own word, read with
+ * pa_read_device_error). The kernel then returns normally: no fault, no hang, the context stays
+ * usable. Returns PA_ERR_INVALID_ARG for a timeout out of range, PA_ERR_CUDA if the launch fails. */
+int pa_selftest_bounded_wait(int32_t timeout_us, int32_t* error_word, void* stream);
+
 /* ---------------------------------------------------------------------------------------------
  * Host block allocator: free list of physical block ids with reference counts.
  * Source: vLLM notes page, "PagedAttention / Block Manager" (O(1) allocation and release with a

@@ -89,6 +89,7 @@ def _load() -> ctypes.CDLL:
         "pa_last_error": (ctypes.c_char_p, []),
         "pa_read_device_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), ctypes.c_int]),
         "pa_version": (ctypes.c_char_p, []),
+        "pa_selftest_bounded_wait": (ctypes.c_int, [I32, ctypes.c_void_p, VP]),
         "pa_allocator_create": (VP, [I32, i32p]),
         "pa_allocator_destroy": (None, [VP]),
         "pa_block_alloc": (I32, [VP]),
@@ -263,6 +264,18 @@ def pa_prefill(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cach
             as_pa_tensor(query_start, "query_start"), as_pa_tensor(context_lens, "context_lens")]
     _check(_lib.pa_prefill(*[ctypes.byref(a) for a in args], int(max_query_len), float(scale), int(num_kv_heads),
                            int(kernel), ctypes.c_void_p(_stream_handle(stream))), "pa_prefill")
+
+
+def pa_selftest_bounded_wait(timeout_us: int, error_word: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Run the library's bounded barrier wait against a barrier nothing arrives on (see include/pa.h):
+    it gives up after timeout_us and sets PA_DEVERR_TIMEOUT in error_word (or the library's word)."""
+    ptr = None
+    if error_word is not None:
+        if not error_word.is_cuda or error_word.dtype != torch.int32:
+            raise ValueError("error_word must be a CUDA int32 tensor")
+        ptr = error_word.data_ptr()
+    _check(_lib.pa_selftest_bounded_wait(int(timeout_us), ctypes.c_void_p(ptr), ctypes.c_void_p(_stream_handle(stream))),
+           "pa_selftest_bounded_wait")
 
 
 # Size of the library's built-in scratch array used by pa_decode_no_alloc (PA_NO_ALLOC_SCRATCH_BYTES).

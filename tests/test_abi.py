@@ -198,3 +198,8 @@ def test_prefill_kernel_choice_is_checked_on_the_host():
     assert lib.pa_prefill(*args, T, 0.125, Hkv, 1, None) == pa.PA_ERR_UNSUPPORTED
     assert "tcgen05" in pa.pa_last_error()
     assert lib.pa_prefill(*args, T, 0.125, Hkv, 5, None) == pa.PA_ERR_INVALID_ARG
+
+
+def test_bounded_wait_selftest_checks_its_timeout_on_the_host():
+    assert pa.lib().pa_selftest_bounded_wait(0, None, None) == pa.PA_ERR_INVALID_ARG
+    assert pa.lib().pa_selftest_bounded_wait(2000000, None, None) == pa.PA_ERR_INVALID_ARG
