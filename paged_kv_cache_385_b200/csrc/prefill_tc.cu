@@ -56,10 +56,10 @@ enum {
   kVFull0 = 7,   // kVStages
   kVEmpty0 = 9,  // kVStages
   kSFull0 = 11,  // 2
-  kPFull = 13,
-  kODone = 14,
-  kAllDone = 15,
-  kTmemSlot = 16,
+  kPFull0 = 13,  // 2: block j arrives on kPFull0 + (j & 1)
+  kODone = 15,
+  kAllDone = 16,
+  kTmemSlot = 17,
 };
 static_assert(8 * (kTmemSlot + 1) <= 256, "barrier area");
 // O is rescaled only when a row's running max grows by more than this (log2 units); until then P and
@@ -141,7 +141,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     mbar_init(B(kSFull0), 1);
     mbar_init(B(kSFull0 + 1), 1);
-    mbar_init(B(kPFull), 4);
+    mbar_init(B(kPFull0), 4);
+    mbar_init(B(kPFull0 + 1), 4);
     mbar_init(B(kODone), 1);
     mbar_init(B(kAllDone), 1);
     fence_barrier_init();
@@ -236,7 +237,9 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (lane == 0) {
       constexpr uint32_t idesc_pv = tc05::idesc_f16(kBf16, kRows, kD, false, true);
       for (int j = 0; j < nkb && ok; ++j) {
-        if (!mbar_wait_bounded(B(kPFull), j & 1, deadline) ||
+        // P_full is two barriers by block parity: block j + 2 cannot arrive before this wait has seen
+        // block j (its QK needs P(j).V), so a parity wait never meets a barrier two phases ahead.
+        if (!mbar_wait_bounded(B(kPFull0 + (j & 1)), (j >> 1) & 1, deadline) ||
             !mbar_wait_bounded(B(kVFull0 + j % kVStages), (j / kVStages) & 1, deadline)) {
           ok = false;
           break;
@@ -363,7 +366,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
       tc05::fence_before_sync();
       __syncwarp();
-      if (lane == 0) mbar_arrive(B(kPFull));
+      if (lane == 0) mbar_arrive(B(kPFull0 + (j & 1)));
     }
     // Epilogue: O / l -> out rows, or (prefix) the row's (m, l, O) -> its workspace slot.
     if (ok) {
