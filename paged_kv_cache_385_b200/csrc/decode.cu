@@ -524,13 +524,22 @@ __global__ void __launch_bounds__(Cfg<KV, QT, D, NT, KIND, OCC>::kThreads, Cfg<K
   }
 
   // pa_decode_step: the CTA holding the sequence's last partition writes head hk's new K/V row
-  // (position ctx - 1) into its slot before any of its page copies start. No other CTA reads that
-  // page, and the proxy fence + barrier order the writes before this CTA's TMA loads.
-  if (p.new_k != nullptr && part == max(nparts, 1) - 1) {
-    const int64_t slot = p.new_slots[s];
+  // (position ctx - 1) into its slot; the proxy fence + barrier order the writes before any TMA load
+  // of that page. The copies of this CTA's first pages are issued before the write (all but a page
+  // in the slot's block), so the write's latency overlaps theirs.
+  const bool fused_here = p.new_k != nullptr && part == max(nparts, 1) - 1;
+  int64_t new_slot = -1;
+  bool do_write = false;
+  if (fused_here) {
+    new_slot = p.new_slots[s];
     // With a shared prefix the new token must lie past it (prefix blocks are read-only here).
     const bool writable = start == 0 || nparts > 0;
-    if (writable && slot >= 0 && slot < static_cast<int64_t>(p.num_blocks) * 16) {
+    do_write = writable && new_slot >= 0 && new_slot < static_cast<int64_t>(p.num_blocks) * 16;
+    if (!do_write && new_slot != -1 && threadIdx.x == 0) atomicOr(p.err, 2u);
+  }
+  auto write_new_token = [&]() {
+    const int64_t slot = new_slot;
+    if (do_write) {
       constexpr int kChunks = D / 8;  // 16-byte input chunks per row
       for (int c = threadIdx.x; c < 2 * kChunks; c += C::kThreads) {
         const bool is_v = c >= kChunks;
@@ -556,11 +565,10 @@ __global__ void __launch_bounds__(Cfg<KV, QT, D, NT, KIND, OCC>::kThreads, Cfg<K
         }
       }
       fence_proxy_async_global();
-    } else if (slot != -1 && threadIdx.x == 0) {
-      atomicOr(p.err, 2u);
     }
     __syncthreads();
-  }
+  };
+  if (fused_here && span == 0) write_new_token();
 
   typedef uint16_t out_t;
   if (span == 0) prefix_check();
@@ -677,7 +685,19 @@ __global__ void __launch_bounds__(Cfg<KV, QT, D, NT, KIND, OCC>::kThreads, Cfg<K
   }
 
   const uint64_t deadline = globaltimer_ns() + 2000000000ull;
-  for (int i = 0; i < min(C::kStages, n_w); ++i) issue(i);
+  // First pages: a page in the new token's block waits until the token is written.
+  const int wblk = do_write && span > 0 ? static_cast<int>(new_slot >> 4) : -1;
+  uint32_t deferred = 0;
+  for (int i = 0; i < min(C::kStages, n_w); ++i) {
+    if (wblk >= 0 && __shfl_sync(kFull, my_bid, i & 31) == wblk) {
+      deferred |= 1u << i;
+    } else {
+      issue(i);
+    }
+  }
+  if (fused_here && span > 0) write_new_token();
+  for (int i = 0; i < min(C::kStages, n_w); ++i)
+    if (deferred & (1u << i)) issue(i);
   bool ok = true;
   int i = 0;
   for (; i < n_w; ++i) {
