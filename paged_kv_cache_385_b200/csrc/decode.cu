@@ -14,7 +14,7 @@
 // for the G query heads of hk (GQA/MQA packing: every K/V byte is read once per KV head); the
 // warps are merged in fixed order through shared memory. With one partition the CTA writes the
 // output; otherwise it writes (acc, m, l) to the workspace and reduce_kernel merges the partitions
-// of a (sequence, head) in index order. No float atomics: the result depends only on logical
+// of a (sequence, head) in a fixed order. No float atomics: the result depends only on logical
 // positions, so permuting physical blocks leaves it bit-identical.
 //
 // Per-page math has two variants:
@@ -22,7 +22,7 @@
 //    (tokens on M, the query group on N), P^T moved into B-fragment layout with movmatrix, then
 //    O^T[D x 8g] += V^T[D x 16] . P^T. K/V fragments come from ldmatrix (V transposed by
 //    ldmatrix.trans); e4m3 pages are widened to f16 in registers (exact).
-//  * CUDA-core (kernel 0): float32 FMA dot products and axpys, for comparison and for G = 1.
+//  * CUDA-core (kernel 0): float32 FMA dot products and axpys, kept for comparison (opts.kernel 0).
 #include <cfloat>
 #include <utility>
 
