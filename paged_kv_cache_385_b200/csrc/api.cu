@@ -2,6 +2,7 @@
 // Host code only; the kernels live in decode.cu and cache.cu.
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -133,13 +134,19 @@ int encode_q_map(CUtensorMap* map, const pa_tensor* q, int group) {
   return PA_OK;
 }
 
+// The device address of the library's error word, looked up once per device. Threads may race on
+// the first lookup; they all store the same address, and the slots are atomics so that is well defined.
 uint32_t* library_error_word() {
-  static uint32_t* words[64] = {nullptr};
+  static std::atomic<uint32_t*> words[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return nullptr;
   if (dev >= 64) return pa::decode_error_word();
-  if (!words[dev]) words[dev] = pa::decode_error_word();
-  return words[dev];
+  uint32_t* w = words[dev].load(std::memory_order_acquire);
+  if (!w) {
+    w = pa::decode_error_word();
+    if (w) words[dev].store(w, std::memory_order_release);
+  }
+  return w;
 }
 
 // Split only when the batch alone cannot fill the GPU: with B * Hkv work units of up to 2048 tokens
