@@ -394,49 +394,81 @@ def run_ours(args, rank, world, local_rank):
     # The step's inputs (q, new K/V, slots, block tables, context lengths) are packed into one pinned
     # host buffer and copied with one H2D copy into a device buffer the step's tensors view; the
     # output comes back with one D2H copy. The KV pool is the resident cache and is not copied.
+    # Inputs and outputs are double-buffered: a copy stream moves step k + 2's inputs in and step k's
+    # output out while the kernels of step k + 1 run, so every step's copies are inside the timed
+    # region without stalling the kernels. The last output read back is checked bit for bit against
+    # the device-timed run's output (same inputs, so the same result).
     e2e = None
     if not args.no_e2e:
+        ref_out = st.out.clone()
         parts = [st.q, st.new_k, st.new_v, st.new_slots, st.bt, st.lens]
         offs, total = [], 0
         for t in parts:
             offs.append(total)
             total += -(-(t.numel() * t.element_size()) // 256) * 256
         hbuf = torch.empty(total, dtype=torch.uint8).pin_memory()
-        dbuf = torch.empty(total, dtype=torch.uint8, device=device)
-        views = []
+        dbufs = [torch.empty(total, dtype=torch.uint8, device=device) for _ in range(2)]
+        views = [[], []]
         for t, o in zip(parts, offs):
             n = t.numel() * t.element_size()
-            hv = hbuf[o:o + n].view(t.dtype).view(t.shape)
-            hv.copy_(t.cpu())
-            views.append(dbuf[o:o + n].view(t.dtype).view(t.shape))
-        st.q, st.new_k, st.new_v, st.new_slots, st.bt, st.lens = views
-        hout = torch.empty(st.out.shape, dtype=st.out.dtype).pin_memory()
-        h2d, d2h = total, hout.numel() * hout.element_size()
+            hbuf[o:o + n].view(t.dtype).view(t.shape).copy_(t.cpu())
+            for b in range(2):
+                views[b].append(dbufs[b][o:o + n].view(t.dtype).view(t.shape))
+        outs = [torch.empty_like(st.out) for _ in range(2)]
+        houts = [torch.empty(st.out.shape, dtype=st.out.dtype).pin_memory() for _ in range(2)]
+        h2d, d2h = total, houts[0].numel() * houts[0].element_size()
         Ke = max(10, min(K, 500))
+        comp = torch.cuda.current_stream(device)
+        copy = torch.cuda.Stream(device)
+        ev_in = [torch.cuda.Event() for _ in range(2)]    # inputs of buffer b landed
+        ev_done = [torch.cuda.Event() for _ in range(2)]  # kernels that used buffer b finished
+        ev_out = [torch.cuda.Event() for _ in range(2)]   # output b read back
 
-        def e2e_step():
-            dbuf.copy_(hbuf, non_blocking=True)
-            st.step()
-            hout.copy_(st.out, non_blocking=True)
+        def h2d_into(b):
+            with torch.cuda.stream(copy):
+                dbufs[b].copy_(hbuf, non_blocking=True)
+                ev_in[b].record(copy)
 
-        for _ in range(3):
-            e2e_step()
+        def run(n_steps, start_ev=None):
+            copy.wait_stream(comp)  # start after everything queued so far (and the start event)
+            h2d_into(0)
+            h2d_into(1)
+            for k in range(n_steps):
+                b = k & 1
+                comp.wait_event(ev_in[b])
+                if k >= 2:
+                    comp.wait_event(ev_out[b])  # output b of step k - 2 has been read back
+                st.q, st.new_k, st.new_v, st.new_slots, st.bt, st.lens = views[b]
+                st.out = outs[b]
+                st.step()
+                ev_done[b].record(comp)
+                with torch.cuda.stream(copy):
+                    copy.wait_event(ev_done[b])
+                    houts[b].copy_(outs[b], non_blocking=True)
+                    ev_out[b].record(copy)
+                    if k + 2 < n_steps:
+                        dbufs[b].copy_(hbuf, non_blocking=True)  # step k + 2's inputs (buffer b is free)
+                        ev_in[b].record(copy)
+            comp.wait_stream(copy)  # the last read-backs are part of the region
+
+        run(3)
         barrier()
         torch.cuda.synchronize(device)
         s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        s0.record()
-        for _ in range(Ke):
-            e2e_step()
-        s1.record()
+        s0.record(comp)
+        run(Ke)
+        s1.record(comp)
         torch.cuda.synchronize(device)
         barrier()
         e_ms = max_over_ranks(s0.elapsed_time(s1), device)
+        same = torch.equal(houts[(Ke - 1) & 1].view(torch.int16), ref_out.cpu().view(torch.int16))
         e2e = {"value": round(job_throughput(kv_bytes, world, e_ms / Ke), 1), "unit": "GB/s",
                "ms_per_step": round(e_ms / Ke, 5), "steps": Ke, "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": d2h,
+               "d2h_bytes_per_step": d2h, "output_matches_device_run": bool(same),
                "note": "per step: one pinned H2D copy of the packed inputs (q, new K/V, slots, block tables, "
-                       "context lens), the decode step through the C ABI, one D2H copy of out; the KV pool "
-                       "is the resident cache"}
+                       "context lens), the decode step through the C ABI, one D2H copy of out; inputs and "
+                       "outputs double-buffered so the copies of neighbouring steps overlap the kernels; the "
+                       "KV pool is the resident cache"}
 
     if world > 1:
         import torch.distributed as dist
