@@ -449,8 +449,6 @@ static int decode_impl(pa_tensor* out, const pa_tensor* q, const pa_tensor* k_ca
   p.always_partials = cascade ? 1 : 0;
   p.merge_prefix_inline = cascade && P == 1 ? 1 : 0;
   p.late_dependency_wait = cascade ? 1 : 0;
-  p.err = opts.error_word ? reinterpret_cast<uint32_t*>(opts.error_word) : library_error_word();
-  if (!p.err) return fail(PA_ERR_CUDA, "no device error word (no current CUDA device?)");
   if (ws_parts > 1) {
     size_t ml_off = 0;
     const size_t need = workspace_layout(B, Hq, D, ws_parts, &ml_off);
@@ -499,6 +497,9 @@ static int decode_impl(pa_tensor* out, const pa_tensor* q, const pa_tensor* k_ca
     p.v_inv_scale = cd == PA_E4M3 ? one / v_scale : 1.0f;
   }
 
+  // Every argument check is above: the first device call is the error word's lookup.
+  p.err = opts.error_word ? reinterpret_cast<uint32_t*>(opts.error_word) : library_error_word();
+  if (!p.err) return fail(PA_ERR_CUDA, "no device error word (no current CUDA device?)");
   CUtensorMap km, vm;
   const int esz = elem_bytes(cd);
   if ((st = encode_pool_map(&km, k_cache, esz)) || (st = encode_pool_map(&vm, v_cache, esz))) return st;

@@ -203,3 +203,35 @@ def test_prefill_kernel_choice_is_checked_on_the_host():
 def test_bounded_wait_selftest_checks_its_timeout_on_the_host():
     assert pa.lib().pa_selftest_bounded_wait(0, None, None) == pa.PA_ERR_INVALID_ARG
     assert pa.lib().pa_selftest_bounded_wait(2000000, None, None) == pa.PA_ERR_INVALID_ARG
+
+
+def test_decode_argument_errors_are_reported_before_device_work():
+    """Every argument error of pa_decode is found on the host, the workspace check included: the
+    tensors here are host memory, so a call that reached the device would not return these codes."""
+    B, Hq, Hkv, D, NB = 2, 8, 2, 128, 16
+    q = _aligned_zeros((B, Hq, D), torch.bfloat16)
+    kc = _aligned_zeros((NB, Hkv, 16, D), torch.bfloat16)
+    kc16 = _aligned_zeros((NB, Hkv, 16, D), torch.float16)
+    bt = torch.zeros(B, 64, dtype=torch.int32)
+    lens = torch.full((B,), 1000, dtype=torch.int32)
+    lib = pa.lib()
+
+    def call(kcache=kc, tables=bt, hkv=Hkv, **kw):
+        ts = [pa.as_pa_tensor(t, n, device=False) for t, n in ((q, "out"), (q, "q"), (kcache, "k"), (kcache, "v"),
+                                                                (tables, "bt"), (lens, "lens"))]
+        opts = pa.PaDecodeOpts()
+        lib.pa_decode_opts_init(ctypes.byref(opts))
+        for k, v in kw.items():
+            setattr(opts, k, v)
+        return lib.pa_decode(*[ctypes.byref(t) for t in ts], 0.088, hkv, ctypes.byref(opts), None)
+
+    assert call(kcache=kc16) == pa.PA_ERR_INVALID_ARG  # f16 cache with a bf16 query
+    assert call(hkv=4) == pa.PA_ERR_INVALID_ARG  # does not match the cache's head count
+    assert call(tables=bt.to(torch.int64)) == pa.PA_ERR_INVALID_ARG
+    assert call(partition_tokens=24) == pa.PA_ERR_INVALID_ARG
+    assert call(kernel=3) == pa.PA_ERR_INVALID_ARG
+    # A split into 1024 / 256 = 4 partitions needs a workspace; none given.
+    assert call(partition_tokens=256) == pa.PA_ERR_WORKSPACE
+    assert "workspace" in pa.pa_last_error()
+    small = _aligned_zeros((64,), torch.uint8)
+    assert call(partition_tokens=256, workspace=small.data_ptr(), workspace_bytes=64) == pa.PA_ERR_WORKSPACE
