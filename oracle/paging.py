@@ -104,8 +104,8 @@ def build_block_tables(context_lens: Sequence[int], order: Sequence[int], num_bl
 
     Sequences are served in order; each takes ceil(ctx / block_size) blocks,
     one ``alloc`` per logical block. With a shared prefix (a whole number of
-    blocks), the first sequence allocates the prefix blocks and every later
-    sequence points its first entries at them (``incref``).
+    blocks), prefix block j is allocated by the first sequence that reaches it
+    and every later sequence reaching it points its entry j at it (``incref``).
     """
     lens = [int(c) for c in context_lens]
     assert shared_prefix_tokens % block_size == 0
@@ -119,7 +119,7 @@ def build_block_tables(context_lens: Sequence[int], order: Sequence[int], num_bl
     for s, nb in enumerate(need):
         for j in range(nb):
             if j < n_prefix:
-                if s == 0:
+                if j == len(prefix_blocks):
                     b = fl.alloc()
                     assert b is not None, "pool exhausted"
                     prefix_blocks.append(b)

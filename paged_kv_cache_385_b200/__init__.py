@@ -427,27 +427,25 @@ def build_block_tables(alloc: BlockAllocator, context_lens: Sequence[int], max_b
                        shared_prefix_tokens: int = 0) -> torch.Tensor:
     """Host int32 block tables [num_seqs, max_blocks] (-1 padded) from the allocator.
 
-    Sequences are served in order, one allocation per logical block; with a shared prefix (a whole
-    number of blocks) the first sequence allocates the prefix blocks and every later sequence takes
-    a reference to them.
+    Sequences are served in order, one allocation per logical block. With a shared prefix (a whole
+    number of blocks) each prefix block is allocated by the first sequence that reaches it, and
+    every later sequence reaching it takes a reference to it.
     """
     if shared_prefix_tokens % BLOCK_SIZE:
         raise ValueError("shared_prefix_tokens must be a multiple of 16")
     npre = shared_prefix_tokens // BLOCK_SIZE
     lens = [int(c) for c in context_lens]
     bt = torch.full((len(lens), max_blocks), -1, dtype=torch.int32)
-    prefix = None
+    prefix = torch.empty(0, dtype=torch.int32)  # prefix blocks allocated so far
     for s, n in enumerate(lens):
         nb = -(-n // BLOCK_SIZE)
         if nb > max_blocks:
             raise ValueError(f"sequence {s} needs {nb} blocks > max_blocks {max_blocks}")
-        shared = min(npre, nb)
-        if s == 0 or shared == 0:
-            row = alloc.alloc_n(nb)
-            if s == 0:
-                prefix = row[:npre].clone()
-        else:
-            alloc.incref_n(prefix[:shared])
-            row = torch.cat([prefix[:shared], alloc.alloc_n(nb - shared)])
+        reuse = min(npre, nb, prefix.numel())
+        if reuse:
+            alloc.incref_n(prefix[:reuse])
+        row = torch.cat([prefix[:reuse], alloc.alloc_n(nb - reuse)])
+        if min(npre, nb) > prefix.numel():
+            prefix = row[:min(npre, nb)].clone()
         bt[s, :nb] = row
     return bt

@@ -235,3 +235,21 @@ def test_decode_argument_errors_are_reported_before_device_work():
     assert "workspace" in pa.pa_last_error()
     small = _aligned_zeros((64,), torch.uint8)
     assert call(partition_tokens=256, workspace=small.data_ptr(), workspace_bytes=64) == pa.PA_ERR_WORKSPACE
+
+
+def test_shared_prefix_blocks_come_from_the_first_sequence_reaching_them():
+    """Sequences shorter than the shared prefix: prefix block j is allocated by the first sequence
+    that needs it and referenced by every later one, as the oracle's free-list model builds it."""
+    lens, npre, nb = [20, 70, 5, 0, 100, 33], 4, 64
+    order = np.random.default_rng(8).permutation(nb)
+    alloc = pa.BlockAllocator(nb, order.tolist())
+    bt = pa.build_block_tables(alloc, lens, 7, shared_prefix_tokens=16 * npre)
+    want = paging.build_block_tables(lens, order, nb, 16, 16 * npre, 7)
+    assert np.array_equal(bt.numpy(), want)
+    need = [-(-n // 16) for n in lens]
+    for j in range(npre):
+        holders = [s for s in range(len(lens)) if need[s] > j]
+        assert len({int(bt[s, j]) for s in holders}) == 1
+        assert alloc.refcount(int(bt[holders[0], j])) == len(holders)
+    distinct = {int(b) for b in bt.flatten().tolist() if b >= 0}
+    assert alloc.num_free == nb - len(distinct)
