@@ -1,5 +1,6 @@
 // C-ABI entry points of libpagedattn: argument validation, TMA descriptor encoding, dispatch.
-// Host code only; the kernels live in decode.cu and cache.cu.
+// Host code only. Every argument error is found here before the first device call; the kernels
+// live in decode.cu, multiquery.cu, prefill_tc.cu, cache.cu and selftest.cu.
 #include <cudaTypedefs.h>
 
 #include <atomic>
