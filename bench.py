@@ -2,8 +2,10 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
 
-A step is the whole hot path for one batch: ``pa_reshape_and_cache`` of the batch's new tokens,
-then ``pa_decode`` (its decode kernel, plus the partition-merge kernel when the context is split).
+A step is the whole hot path for one batch: the write of the batch's new tokens into their slots
+and the decode attention over every sequence's pages (plus the partition merge when the context is
+split). By default (``--step fused``) both run in one launch, ``pa_decode_step``; ``--step separate``
+calls ``pa_reshape_and_cache`` then ``pa_decode``; ``--step cascade`` calls ``pa_decode_cascade``.
 The default workload is the Llama-7B-shaped MHA batch: 32 sequences x 2048 tokens, 32 query = 32 KV
 heads, head_dim 128, fp16, 16-token blocks scattered through a 5120-block pool. Its KV cache
 (1.07 GB per step) is far larger than L2 (126 MB), so no L2 flush is needed between steps.
