@@ -22,9 +22,11 @@
  *     never allocates, frees or synchronises on pa_reshape_and_cache/pa_decode.
  *     Work is enqueued on the caller's stream (a cudaStream_t passed as void*;
  *     NULL = the legacy default stream). Calls return after enqueueing.
- *   - Host-side validation runs before any launch and returns a negative
+ *   - Host-side validation (shapes, dtypes, strides, alignment, options, the
+ *     workspace size) runs before any CUDA call and returns a negative
  *     pa_status without touching device memory; pa_last_error() then gives a
- *     one-line reason (thread-local). A launch failure returns PA_ERR_CUDA.
+ *     one-line reason (thread-local). A failed CUDA call or launch returns
+ *     PA_ERR_CUDA.
  *   - Conditions only the device can see (a block id or slot outside the pool,
  *     a context longer than max_context_len, a pipeline wait that timed out)
  *     never fault: the offending page or token is skipped and a bit is OR-ed
