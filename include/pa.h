@@ -250,9 +250,11 @@ size_t pa_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t 
  * be NULL and workspace_bytes 0, else PA_ERR_INVALID_ARG). All other arguments, results and errors
  * are those of pa_decode.
  *   - A batch whose split needs more than PA_NO_ALLOC_SCRATCH_BYTES (see pa_decode_workspace_bytes)
- *     is rejected with PA_ERR_WORKSPACE before any device work; larger partition_tokens needs less.
- *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress, with
- *     that device current) and caches it; make that first call before any stream capture.
+ *     is rejected with PA_ERR_WORKSPACE before any CUDA call, like every other argument error;
+ *     larger partition_tokens needs less.
+ *   - The first call on a device that splits a context looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current), after its argument checks, and caches it;
+ *     make such a call before any stream capture.
  *   - The array takes PA_NO_ALLOC_SCRATCH_BYTES (32 MiB) on every device where the library's device
  *     code is loaded (depending on CUDA's module-loading mode, at start-up or at the latest on the
  *     first call), until the process exits.

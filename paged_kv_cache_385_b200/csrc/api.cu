@@ -313,7 +313,8 @@ int pa_reshape_and_cache(const pa_tensor* key, const pa_tensor* value, const pa_
 static int decode_impl(pa_tensor* out, const pa_tensor* q, const pa_tensor* k_cache, const pa_tensor* v_cache,
                        const pa_tensor* block_tables, const pa_tensor* context_lens, float scale, int32_t num_kv_heads,
                        const pa_decode_opts* opts_in, void* stream, const pa_tensor* new_key,
-                       const pa_tensor* new_value, const pa_tensor* new_slots, int32_t prefix_tokens = 0) {
+                       const pa_tensor* new_value, const pa_tensor* new_slots, int32_t prefix_tokens = 0,
+                       const pa::BuiltinScratch* builtin = nullptr) {
   pa_decode_opts opts;
   pa_decode_opts_init(&opts);
   if (opts_in) opts = *opts_in;
@@ -395,7 +396,7 @@ static int decode_impl(pa_tensor* out, const pa_tensor* q, const pa_tensor* k_ca
   if (pt < 0 || pt % 16 || pt > pa::kMaxPartitionTokens)
     return fail(PA_ERR_INVALID_ARG, "partition_tokens %lld must be a multiple of 16 in [0, %d]", (long long)pt,
                 pa::kMaxPartitionTokens);
-  const bool have_ws = opts.workspace != nullptr && opts.workspace_bytes > 0;
+  const bool have_ws = (opts.workspace != nullptr && opts.workspace_bytes > 0) || builtin != nullptr;
   // Cascade: the shared prefix goes to the prefix kernel (n_pre chunks); this grid covers the suffix.
   const bool cascade = prefix_tokens > 0;
   int64_t n_pre = 0;
@@ -450,15 +451,23 @@ static int decode_impl(pa_tensor* out, const pa_tensor* q, const pa_tensor* k_ca
   p.always_partials = cascade ? 1 : 0;
   p.merge_prefix_inline = cascade && P == 1 ? 1 : 0;
   p.late_dependency_wait = cascade ? 1 : 0;
+  size_t ml_off = 0;
   if (ws_parts > 1) {
-    size_t ml_off = 0;
     const size_t need = workspace_layout(B, Hq, D, ws_parts, &ml_off);
-    if (!have_ws || opts.workspace_bytes < need)
-      return fail(PA_ERR_WORKSPACE, "split into %lld partitions needs a workspace of %zu bytes (got %zu)",
-                  (long long)ws_parts, need, have_ws ? opts.workspace_bytes : size_t(0));
-    if (!aligned(opts.workspace, 256)) return fail(PA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
-    p.ws_acc = static_cast<float*>(opts.workspace);
-    p.ws_ml = reinterpret_cast<float*>(static_cast<char*>(opts.workspace) + ml_off);
+    if (builtin) {
+      // The built-in array's address is looked up below, after the last argument check.
+      if (need > builtin->bytes)
+        return fail(PA_ERR_WORKSPACE,
+                    "this batch needs %zu bytes of scratch; the built-in array holds %zu (use pa_decode with a "
+                    "workspace, or larger partition_tokens)", need, builtin->bytes);
+    } else {
+      if (!have_ws || opts.workspace_bytes < need)
+        return fail(PA_ERR_WORKSPACE, "split into %lld partitions needs a workspace of %zu bytes (got %zu)",
+                    (long long)ws_parts, need, have_ws ? opts.workspace_bytes : size_t(0));
+      if (!aligned(opts.workspace, 256)) return fail(PA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+      p.ws_acc = static_cast<float*>(opts.workspace);
+      p.ws_ml = reinterpret_cast<float*>(static_cast<char*>(opts.workspace) + ml_off);
+    }
   }
 
   if (new_key) {
@@ -498,9 +507,17 @@ static int decode_impl(pa_tensor* out, const pa_tensor* q, const pa_tensor* k_ca
     p.v_inv_scale = cd == PA_E4M3 ? one / v_scale : 1.0f;
   }
 
-  // Every argument check is above: the first device call is the error word's lookup.
+  // Every argument check is above: the device calls start here.
   p.err = opts.error_word ? reinterpret_cast<uint32_t*>(opts.error_word) : library_error_word();
   if (!p.err) return fail(PA_ERR_CUDA, "no device error word (no current CUDA device?)");
+  if (builtin && ws_parts > 1) {
+    void* base = nullptr;
+    const cudaError_t le = builtin->lookup(&base);
+    if (le != cudaSuccess || !base)
+      return fail(PA_ERR_CUDA, "address of the built-in scratch array: %s", cudaGetErrorString(le));
+    p.ws_acc = static_cast<float*>(base);
+    p.ws_ml = reinterpret_cast<float*>(static_cast<char*>(base) + ml_off);
+  }
   CUtensorMap km, vm;
   const int esz = elem_bytes(cd);
   if ((st = encode_pool_map(&km, k_cache, esz)) || (st = encode_pool_map(&vm, v_cache, esz))) return st;
@@ -584,6 +601,23 @@ int pa_decode(pa_tensor* out, const pa_tensor* q, const pa_tensor* k_cache, cons
   return decode_impl(out, q, k_cache, v_cache, block_tables, context_lens, scale, num_kv_heads, opts, stream, nullptr,
                      nullptr, nullptr);
 }
+
+}  // extern "C"
+
+namespace pa {
+int decode_with_builtin_scratch(pa_tensor* out, const pa_tensor* q, const pa_tensor* k_cache,
+                                const pa_tensor* v_cache, const pa_tensor* block_tables,
+                                const pa_tensor* context_lens, float scale, int32_t num_kv_heads,
+                                const pa_decode_opts* opts, void* stream, const BuiltinScratch& scratch) {
+  if (opts && (opts->workspace != nullptr || opts->workspace_bytes != 0))
+    return fail(PA_ERR_INVALID_ARG, "no workspace may be given with the built-in scratch (opts.workspace must be "
+                                    "NULL, size 0)");
+  return decode_impl(out, q, k_cache, v_cache, block_tables, context_lens, scale, num_kv_heads, opts, stream, nullptr,
+                     nullptr, nullptr, 0, &scratch);
+}
+}  // namespace pa
+
+extern "C" {
 
 int pa_decode_cascade(pa_tensor* out, const pa_tensor* q, const pa_tensor* key, const pa_tensor* value,
                       const pa_tensor* slot_mapping, pa_tensor* k_cache, pa_tensor* v_cache,

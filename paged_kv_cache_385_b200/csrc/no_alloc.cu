@@ -10,8 +10,8 @@
 // The array (PA_NO_ALLOC_SCRATCH_BYTES) is a file-scope static __device__ object: every device where
 // the library's device code is loaded holds it until the process exits. In host code the array's name is only a
 // host-side stand-in, never a device address, so its address is looked up with
-// cudaGetSymbolAddress once per device, with that device current, on the first call made on that
-// device, and cached. Every call on a device shares the one array, which keeps the last call's
+// cudaGetSymbolAddress once per device, with that device current, on the first call on that device
+// that splits a context (after all of its argument checks), and cached. Every call on a device shares the one array, which keeps the last call's
 // contents; nothing in it has to start at zero, because each call writes every partial result it
 // later reads. Calls whose kernels overlap on the GPU (for example, issued on two streams with no
 // ordering between them) race on the array.
@@ -50,35 +50,10 @@ cudaError_t scratch_on_current_device(void** out) {
 extern "C" int pa_decode_no_alloc(pa_tensor* out, const pa_tensor* q, const pa_tensor* k_cache,
                                   const pa_tensor* v_cache, const pa_tensor* block_tables,
                                   const pa_tensor* context_lens, float scale, int32_t num_kv_heads,
-                                  const pa_decode_opts* opts_in, void* stream) {
-  pa_decode_opts opts;
-  pa_decode_opts_init(&opts);
-  if (opts_in) opts = *opts_in;
-  if (opts.workspace != nullptr || opts.workspace_bytes != 0)
-    return pa::set_last_error(PA_ERR_INVALID_ARG,
-                              "pa_decode_no_alloc takes no workspace (opts.workspace must be NULL, size 0)");
-  // Reject batches whose split would need more scratch than the array holds, before any CUDA call.
-  if (q && block_tables && q->ndim == 3 && block_tables->ndim == 2 && num_kv_heads > 0 && q->shape[0] > 0 &&
-      q->shape[1] > 0 && q->shape[2] > 0 && q->shape[0] <= 0x7fffffff && q->shape[1] <= 0x7fffffff) {
-    const int64_t cap = block_tables->shape[1] * PA_BLOCK_SIZE;
-    int64_t max_ctx = opts.max_context_len > 0 ? opts.max_context_len : cap;
-    if (max_ctx > cap) max_ctx = cap;
-    if (max_ctx > 0x7fffffff) max_ctx = 0x7fffffff;
-    const size_t need = pa_decode_workspace_bytes(
-        static_cast<int32_t>(q->shape[0]), static_cast<int32_t>(q->shape[1]), num_kv_heads,
-        static_cast<int32_t>(q->shape[2]), static_cast<int32_t>(max_ctx), opts.partition_tokens);
-    if (need > PA_NO_ALLOC_SCRATCH_BYTES)
-      return pa::set_last_error(PA_ERR_WORKSPACE,
-                                "pa_decode_no_alloc: this batch needs %zu bytes of scratch; the built-in array "
-                                "holds %zu (use pa_decode with a workspace, or larger partition_tokens)",
-                                need, static_cast<size_t>(PA_NO_ALLOC_SCRATCH_BYTES));
-  }
-  void* scratch = nullptr;
-  const cudaError_t e = scratch_on_current_device(&scratch);
-  if (e != cudaSuccess)
-    return pa::set_last_error(PA_ERR_CUDA, "pa_decode_no_alloc: cudaGetSymbolAddress of the scratch array: %s",
-                              cudaGetErrorString(e));
-  opts.workspace = scratch;
-  opts.workspace_bytes = PA_NO_ALLOC_SCRATCH_BYTES;
-  return pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale, num_kv_heads, &opts, stream);
+                                  const pa_decode_opts* opts, void* stream) {
+  // Every argument check, including whether the batch's split fits the array, runs before the
+  // array's address is looked up (the first CUDA call).
+  const pa::BuiltinScratch scratch{static_cast<size_t>(PA_NO_ALLOC_SCRATCH_BYTES), scratch_on_current_device};
+  return pa::decode_with_builtin_scratch(out, q, k_cache, v_cache, block_tables, context_lens, scale, num_kv_heads,
+                                         opts, stream, scratch);
 }

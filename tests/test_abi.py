@@ -253,3 +253,32 @@ def test_shared_prefix_blocks_come_from_the_first_sequence_reaching_them():
         assert alloc.refcount(int(bt[holders[0], j])) == len(holders)
     distinct = {int(b) for b in bt.flatten().tolist() if b >= 0}
     assert alloc.num_free == nb - len(distinct)
+
+
+def test_no_alloc_decode_checks_arguments_before_the_scratch_lookup():
+    """pa_decode_no_alloc finds argument errors, the scratch capacity included, before its first CUDA
+    call (the lookup of the built-in array): with host tensors it returns them, not PA_ERR_CUDA."""
+    B, Hkv, G, D = 64, 8, 8, 128
+    q = _aligned_zeros((B, Hkv * G, D), torch.bfloat16)
+    kc = _aligned_zeros((16, Hkv, 16, D), torch.bfloat16)
+    kc16 = _aligned_zeros((16, Hkv, 16, D), torch.float16)
+    bt = torch.zeros(B, 8192, dtype=torch.int32)
+    lens = torch.ones(B, dtype=torch.int32)
+    lib = pa.lib()
+
+    def call(kcache=kc, **kw):
+        ts = [pa.as_pa_tensor(t, n, device=False) for t, n in ((q, "out"), (q, "q"), (kcache, "k"), (kcache, "v"),
+                                                                (bt, "bt"), (lens, "lens"))]
+        opts = pa.PaDecodeOpts()
+        lib.pa_decode_opts_init(ctypes.byref(opts))
+        for k, v in kw.items():
+            setattr(opts, k, v)
+        return lib.pa_decode_no_alloc(*[ctypes.byref(t) for t in ts], 0.1, Hkv, ctypes.byref(opts), None)
+
+    assert call(kcache=kc16) == pa.PA_ERR_INVALID_ARG
+    assert call(partition_tokens=24) == pa.PA_ERR_INVALID_ARG
+    # 64 sequences x 64 heads x 512 partitions of 256 tokens: far more than the built-in array.
+    assert call(max_context_len=8192 * 16, partition_tokens=256) == pa.PA_ERR_WORKSPACE
+    assert "scratch" in pa.pa_last_error()
+    small = _aligned_zeros((256,), torch.uint8)
+    assert call(workspace=small.data_ptr(), workspace_bytes=256) == pa.PA_ERR_INVALID_ARG
