@@ -12,6 +12,7 @@
 #include <string>
 
 #include "../../include/pa.h"
+#include "builtin_scratch.h"
 #include "internal.h"
 
 namespace {

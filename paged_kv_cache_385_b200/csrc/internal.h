@@ -142,26 +142,8 @@ cudaError_t launch_copy_blocks(const CopyParams& p, cudaStream_t stream);
 
 uint32_t* decode_error_word();  // device address of the library's own error word
 
-// Split-partition scratch owned by the library (pa_decode_no_alloc): its size, checked against the
-// batch's need with the other arguments, and the lookup of its device address on the current
-// device, made only after every argument check has passed.
-struct BuiltinScratch {
-  size_t bytes;
-  cudaError_t (*lookup)(void** device_address);
-};
-
 // Record the reason pa_last_error() reports for this thread; returns status.
 int set_last_error(int status, const char* fmt, ...);
 cudaError_t read_and_clear_error_word(uint32_t* bits, int clear);
 
-}  // namespace pa
-
-struct pa_tensor;
-struct pa_decode_opts;
-namespace pa {
-// pa_decode with its split scratch taken from `scratch` instead of opts.workspace (which must be NULL).
-int decode_with_builtin_scratch(pa_tensor* out, const pa_tensor* q, const pa_tensor* k_cache,
-                                const pa_tensor* v_cache, const pa_tensor* block_tables,
-                                const pa_tensor* context_lens, float scale, int32_t num_kv_heads,
-                                const pa_decode_opts* opts, void* stream, const BuiltinScratch& scratch);
 }  // namespace pa

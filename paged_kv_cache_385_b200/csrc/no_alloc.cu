@@ -18,6 +18,7 @@
 #include <mutex>
 
 #include "../../include/pa.h"
+#include "builtin_scratch.h"
 #include "internal.h"
 
 namespace {
