@@ -325,7 +325,9 @@ int32_t pa_allocator_num_blocks(const pa_allocator* a);
 /* Allocate n blocks into out[0..n) all-or-nothing: PA_ERR_EXHAUSTED (nothing taken) if fewer
  * than n are free. */
 int pa_blocks_alloc_n(pa_allocator* a, int32_t n, int32_t* out);
-/* incref / free each of blocks[0..n); stops at the first bad id and returns its error. */
+/* incref / free each of blocks[0..n) (an id may repeat: it is counted once per listing),
+ * all-or-nothing: if any id is not allocated, would be freed more often than it is referenced
+ * (PA_ERR_BAD_BLOCK) or would overflow its count (PA_ERR_INVALID_ARG), nothing changes. */
 int pa_blocks_incref_n(pa_allocator* a, int32_t n, const int32_t* blocks);
 int pa_blocks_free_n(pa_allocator* a, int32_t n, const int32_t* blocks);
 

@@ -10,6 +10,7 @@
 // block released most recently is reused first (warm in L2). Copy-on-write (前世今生 §3.2): a
 // sequence about to write into a block other sequences share moves its reference to a fresh block,
 // whose page the caller fills with pa_copy_blocks first. No GPU is involved.
+#include <algorithm>
 #include <cstdint>
 #include <new>
 #include <vector>
@@ -20,6 +21,35 @@ struct pa_allocator {
   std::vector<int32_t> stack;  // free ids; top = back
   std::vector<int32_t> ref;    // 0 = free
 };
+
+namespace {
+
+// Whether changing the count of every listed block by `delta` (+1 or -1) once per listing keeps all
+// counts valid: every id allocated, no block freed more often than it is referenced, no count past
+// INT32_MAX. Nothing is changed; a block listed k times is checked against k changes.
+int check_batch(const pa_allocator* a, int32_t n, const int32_t* blocks, int delta) {
+  std::vector<int32_t> ids;
+  try {
+    ids.assign(blocks, blocks + n);
+  } catch (...) {
+    return PA_ERR_INVALID_ARG;
+  }
+  std::sort(ids.begin(), ids.end());
+  const int32_t num_blocks = static_cast<int32_t>(a->ref.size());
+  for (size_t i = 0; i < ids.size();) {
+    const int32_t b = ids[i];
+    size_t j = i;
+    while (j < ids.size() && ids[j] == b) ++j;
+    const int64_t times = static_cast<int64_t>(j - i);
+    if (b < 0 || b >= num_blocks || a->ref[b] == 0) return PA_ERR_BAD_BLOCK;
+    if (delta < 0 && times > a->ref[b]) return PA_ERR_BAD_BLOCK;
+    if (delta > 0 && a->ref[b] + times > INT32_MAX) return PA_ERR_INVALID_ARG;
+    i = j;
+  }
+  return PA_OK;
+}
+
+}  // namespace
 
 extern "C" {
 
@@ -109,21 +139,20 @@ int pa_blocks_alloc_n(pa_allocator* a, int32_t n, int32_t* out) {
   return PA_OK;
 }
 
+// Both batch calls are all-or-nothing: the whole list is checked first, then applied in list order
+// (so blocks whose last reference goes are pushed in that order, as n single frees would).
 int pa_blocks_incref_n(pa_allocator* a, int32_t n, const int32_t* blocks) {
   if (!a || n < 0 || (n > 0 && !blocks)) return PA_ERR_INVALID_ARG;
-  for (int32_t i = 0; i < n; ++i) {
-    const int r = pa_block_incref(a, blocks[i]);
-    if (r != PA_OK) return r;
-  }
+  if (const int r = check_batch(a, n, blocks, +1)) return r;
+  for (int32_t i = 0; i < n; ++i) ++a->ref[blocks[i]];
   return PA_OK;
 }
 
 int pa_blocks_free_n(pa_allocator* a, int32_t n, const int32_t* blocks) {
   if (!a || n < 0 || (n > 0 && !blocks)) return PA_ERR_INVALID_ARG;
-  for (int32_t i = 0; i < n; ++i) {
-    const int r = pa_block_free(a, blocks[i]);
-    if (r != PA_OK) return r;
-  }
+  if (const int r = check_batch(a, n, blocks, -1)) return r;
+  for (int32_t i = 0; i < n; ++i)
+    if (--a->ref[blocks[i]] == 0) a->stack.push_back(blocks[i]);
   return PA_OK;
 }
 

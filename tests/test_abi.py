@@ -1,5 +1,6 @@
 """CPU checks of the C-ABI library: it loads, exports every declared entry point, and its host-side
 allocator and slot helper agree with the oracle's models. No GPU and no device compute here."""
+import copy
 import ctypes
 import os
 import re
@@ -282,3 +283,32 @@ def test_no_alloc_decode_checks_arguments_before_the_scratch_lookup():
     assert "scratch" in pa.pa_last_error()
     small = _aligned_zeros((256,), torch.uint8)
     assert call(workspace=small.data_ptr(), workspace_bytes=256) == pa.PA_ERR_INVALID_ARG
+
+
+@settings(max_examples=120, deadline=None)
+@given(n=st.integers(1, 12), pre=st.lists(st.tuples(st.sampled_from("ai"), st.integers(0, 11)), max_size=30),
+       batch=st.lists(st.integers(-1, 12), max_size=10), free=st.booleans())
+def test_batch_incref_and_free_are_all_or_nothing(n, pre, batch, free):
+    """A batch call equals the same single calls in list order when every one of them would succeed,
+    and otherwise fails and changes nothing (counts, free list and its order)."""
+    a = pa.BlockAllocator(n)
+    model = paging.FreeListModel(n, list(range(n)))
+    for op, b in pre:  # some state: allocated blocks, some shared
+        if op == "a":
+            if model.alloc() is not None:
+                a.alloc()
+        elif model.incref(b):
+            a.incref(b)
+    trial = copy.deepcopy(model)  # the single calls, applied to a copy
+    ok = all((trial.free if free else trial.incref)(b) for b in batch)
+    arr = torch.tensor(batch, dtype=torch.int32)
+    lib = pa.lib()
+    r = (lib.pa_blocks_free_n if free else lib.pa_blocks_incref_n)(a._h, len(batch), pa._i32_ptr(arr))
+    want = trial if ok else model
+    assert (r == pa.PA_OK) == ok
+    if not ok:
+        assert r == pa.PA_ERR_BAD_BLOCK
+    assert [a.refcount(b) for b in range(n)] == [want.refcount(b) for b in range(n)]
+    # The free lists agree in content and order: n allocations drain them identically.
+    got = [lib.pa_block_alloc(a._h) for _ in range(a.num_free)]
+    assert got == [want.alloc() for _ in range(want.num_free)]
