@@ -198,7 +198,8 @@ int pa_decode_cascade(pa_tensor* out, const pa_tensor* q, const pa_tensor* key, 
                       const pa_tensor* block_tables, const pa_tensor* context_lens, int32_t shared_prefix_tokens,
                       float scale, int32_t num_kv_heads, const pa_decode_opts* opts, void* stream);
 
-/* Workspace bytes pa_decode_cascade needs (partition_tokens 0 = the library's choice). Host only. */
+/* Workspace bytes pa_decode_cascade needs (partition_tokens 0 = the library's choice); SIZE_MAX when
+ * the size does not fit in 64 bits. Host only. */
 size_t pa_decode_cascade_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
                                          int32_t head_dim, int32_t max_context_len, int32_t shared_prefix_tokens,
                                          int32_t partition_tokens);
@@ -233,8 +234,8 @@ int pa_prefill(pa_tensor* out, const pa_tensor* q, const pa_tensor* k_cache, con
  * about four CTAs per SM, else 256. Host only. */
 int32_t pa_decode_partition_tokens(int32_t num_seqs, int32_t num_kv_heads, int32_t max_context_len);
 
-/* Workspace bytes pa_decode needs for these sizes (0 when no split happens). partition_tokens 0
- * applies pa_decode_partition_tokens. Host only. */
+/* Workspace bytes pa_decode needs for these sizes (0 when no split happens; SIZE_MAX when the size
+ * does not fit in 64 bits). partition_tokens 0 applies pa_decode_partition_tokens. Host only. */
 size_t pa_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
                                  int32_t max_context_len, int32_t partition_tokens);
 

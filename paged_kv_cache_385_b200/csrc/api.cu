@@ -8,6 +8,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <initializer_list>
 #include <mutex>
 #include <string>
 
@@ -49,6 +50,15 @@ int elem_bytes(int dtype) {
     default:
       return 0;
   }
+}
+
+// Product of non-negative sizes, or -1 when it does not fit in int64 (a descriptor may claim any
+// shape; the checks below must not overflow on it).
+int64_t checked_product(std::initializer_list<int64_t> xs) {
+  int64_t r = 1;
+  for (const int64_t x : xs)
+    if (x < 0 || __builtin_mul_overflow(r, x, &r)) return -1;
+  return r;
 }
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
@@ -160,16 +170,23 @@ int32_t auto_partition_tokens(int32_t num_seqs, int32_t num_kv_heads, int32_t ma
   const int64_t units = static_cast<int64_t>(num_seqs) * num_kv_heads;
   if (max_ctx <= pa::kMaxPartitionTokens && units >= kFillUnits) return 0;
   for (int32_t pt = pa::kMaxPartitionTokens; pt > 256; pt /= 2)
-    if (units * ((max_ctx + pt - 1) / pt) >= kFillUnits && max_ctx > pt) return pt;
+    if (units * ((static_cast<int64_t>(max_ctx) + pt - 1) / pt) >= kFillUnits && max_ctx > pt) return pt;
   return max_ctx > 256 ? 256 : 0;
 }
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // Layout of the split-partition workspace: acc [B, Hq, P, D] floats, then (m, l) [B, Hq, P, 2].
+// SIZE_MAX when the size does not fit in int64 (no buffer can hold it).
 size_t workspace_layout(int64_t B, int64_t Hq, int64_t D, int64_t P, size_t* ml_offset) {
-  const size_t acc = round_up(static_cast<size_t>(B * Hq * P * D) * sizeof(float), 256);
-  const size_t ml = round_up(static_cast<size_t>(B * Hq * P * 2) * sizeof(float), 256);
+  const int64_t acc_bytes = checked_product({B, Hq, P, D, static_cast<int64_t>(sizeof(float))});
+  const int64_t ml_bytes = checked_product({B, Hq, P, 2, static_cast<int64_t>(sizeof(float))});
+  if (acc_bytes < 0 || ml_bytes < 0 || acc_bytes > (INT64_MAX >> 2) || ml_bytes > (INT64_MAX >> 2)) {
+    if (ml_offset) *ml_offset = 0;
+    return SIZE_MAX;
+  }
+  const size_t acc = round_up(static_cast<size_t>(acc_bytes), 256);
+  const size_t ml = round_up(static_cast<size_t>(ml_bytes), 256);
   if (ml_offset) *ml_offset = acc;
   return acc + ml;
 }
@@ -267,6 +284,8 @@ int pa_reshape_and_cache(const pa_tensor* key, const pa_tensor* value, const pa_
     return fail(PA_ERR_INVALID_ARG, "cache shape must be [num_blocks, %lld, 16, %lld]", (long long)Hkv, (long long)D);
   if (!is_contiguous(k_cache) || !is_contiguous(v_cache)) return fail(PA_ERR_INVALID_ARG, "caches must be contiguous");
   if (D % 8 != 0 || D <= 0) return fail(PA_ERR_UNSUPPORTED, "head_dim %lld is not a multiple of 8", (long long)D);
+  if (checked_product({k_cache->shape[0], Hkv, PA_BLOCK_SIZE, D, 2}) < 0)
+    return fail(PA_ERR_UNSUPPORTED, "pool too large (its size does not fit in 64 bits)");
   if (T == 0) return ok();
   if (key->stride[2] != 1 || value->stride[2] != 1) return fail(PA_ERR_INVALID_ARG, "key/value last stride must be 1");
   if (!aligned(key->data, 16) || !aligned(value->data, 16) || key->stride[0] % 8 || key->stride[1] % 8 ||
@@ -354,7 +373,7 @@ static int decode_impl(pa_tensor* out, const pa_tensor* q, const pa_tensor* k_ca
   if (B == 0 || Hq == 0) return ok();
   const int64_t NB = k_cache->shape[0];
   if (NB <= 0) return fail(PA_ERR_INVALID_ARG, "empty pool");
-  if (NB * num_kv_heads * 16 > 0x7fffffffLL) return fail(PA_ERR_UNSUPPORTED, "pool too large (rows exceed 2^31)");
+  if (NB > 0x7fffffffLL / 16 / num_kv_heads) return fail(PA_ERR_UNSUPPORTED, "pool too large (rows exceed 2^31)");
   if (B > 65535 || num_kv_heads > 65535) return fail(PA_ERR_UNSUPPORTED, "num_seqs and num_kv_heads must be <= 65535");
   if (G > 16) return fail(PA_ERR_UNSUPPORTED, "query group %lld > 16", (long long)G);
   if (q->stride[2] != 1 || out->stride[2] != 1) return fail(PA_ERR_INVALID_ARG, "q/out last stride must be 1");
@@ -370,6 +389,8 @@ static int decode_impl(pa_tensor* out, const pa_tensor* q, const pa_tensor* k_ca
     return fail(PA_ERR_INVALID_ARG, "NULL data pointer");
   const int64_t max_blocks = block_tables->shape[1];
   if (max_blocks <= 0) return fail(PA_ERR_INVALID_ARG, "block_tables has no columns");
+  // Tokens a table row can address; contexts are int32, so columns past 2^31 / 16 are never read.
+  const int64_t table_tokens = std::min<int64_t>(max_blocks, 0x7fffffff / 16) * 16;
 
   pa::DecodeConfig cfg{};
   cfg.kv = cd == PA_E4M3 ? pa::KvType::E4M3 : (cd == PA_BF16 ? pa::KvType::BF16 : pa::KvType::F16);
@@ -390,9 +411,9 @@ static int decode_impl(pa_tensor* out, const pa_tensor* q, const pa_tensor* k_ca
       return fail(PA_ERR_INVALID_ARG, "E4M3 cache scales must be finite and > 0");
   }
 
-  int64_t max_ctx = opts.max_context_len > 0 ? opts.max_context_len : max_blocks * 16;
+  int64_t max_ctx = opts.max_context_len > 0 ? opts.max_context_len : table_tokens;
   if (opts.max_context_len < 0) return fail(PA_ERR_INVALID_ARG, "max_context_len < 0");
-  max_ctx = std::min<int64_t>(max_ctx, max_blocks * 16);
+  max_ctx = std::min<int64_t>(max_ctx, table_tokens);
   int64_t pt = opts.partition_tokens;
   if (pt < 0 || pt % 16 || pt > pa::kMaxPartitionTokens)
     return fail(PA_ERR_INVALID_ARG, "partition_tokens %lld must be a multiple of 16 in [0, %d]", (long long)pt,
@@ -405,7 +426,7 @@ static int decode_impl(pa_tensor* out, const pa_tensor* q, const pa_tensor* k_ca
   if (cascade) {
     if (cd == PA_E4M3) return fail(PA_ERR_UNSUPPORTED, "shared-prefix decode takes F16 or BF16 caches");
     if (prefix_tokens % 16) return fail(PA_ERR_INVALID_ARG, "shared_prefix_tokens must be a multiple of 16");
-    if (prefix_tokens > max_blocks * 16)
+    if (prefix_tokens > table_tokens)
       return fail(PA_ERR_INVALID_ARG, "shared_prefix_tokens %d exceeds the block-table width", prefix_tokens);
     n_pre = (prefix_tokens + pa::kPrefixChunkTokens - 1) / pa::kPrefixChunkTokens;
     if (opts.prefix_kernel < -1 || opts.prefix_kernel > 1)
@@ -455,6 +476,8 @@ static int decode_impl(pa_tensor* out, const pa_tensor* q, const pa_tensor* k_ca
   size_t ml_off = 0;
   if (ws_parts > 1) {
     const size_t need = workspace_layout(B, Hq, D, ws_parts, &ml_off);
+    if (need == SIZE_MAX)
+      return fail(PA_ERR_UNSUPPORTED, "split into %lld partitions: the workspace size overflows", (long long)ws_parts);
     if (builtin) {
       // The built-in array's address is looked up below, after the last argument check.
       if (need > builtin->bytes)
@@ -578,7 +601,9 @@ int pa_copy_blocks(pa_tensor* k_cache, pa_tensor* v_cache, const pa_tensor* bloc
   const int64_t N = block_mapping->shape[0];
   if (N == 0) return ok();
   if (N > 0x7fffffff) return fail(PA_ERR_INVALID_ARG, "too many pairs");
-  const int64_t block_bytes = k_cache->shape[1] * 16 * k_cache->shape[3] * elem_bytes(k_cache->dtype);
+  const int64_t block_bytes = checked_product({k_cache->shape[1], 16, k_cache->shape[3], elem_bytes(k_cache->dtype)});
+  if (block_bytes < 0 || checked_product({k_cache->shape[0], block_bytes}) < 0)
+    return fail(PA_ERR_UNSUPPORTED, "pool too large (its size does not fit in 64 bits)");
   if (block_bytes % 16) return fail(PA_ERR_UNSUPPORTED, "block size in bytes must be a multiple of 16");
   if (!aligned(k_cache->data, 16) || !aligned(v_cache->data, 16)) return fail(PA_ERR_INVALID_ARG, "caches must be 16-byte aligned");
   if (!block_mapping->data) return fail(PA_ERR_INVALID_ARG, "NULL data pointer");
@@ -680,7 +705,7 @@ int pa_prefill(pa_tensor* out, const pa_tensor* q, const pa_tensor* k_cache, con
   if (T == 0 || B == 0) return ok();
   if (max_query_len <= 0) return fail(PA_ERR_INVALID_ARG, "max_query_len must be > 0");
   if (B > 65535 || num_kv_heads > 65535) return fail(PA_ERR_UNSUPPORTED, "num_seqs and num_kv_heads must be <= 65535");
-  if (k_cache->shape[0] * num_kv_heads * 16 > 0x7fffffffLL) return fail(PA_ERR_UNSUPPORTED, "pool too large");
+  if (k_cache->shape[0] > 0x7fffffffLL / 16 / num_kv_heads) return fail(PA_ERR_UNSUPPORTED, "pool too large");
   if (q->stride[2] != 1 || out->stride[2] != 1 || !aligned(q->data, 16) || !aligned(out->data, 16) ||
       q->stride[0] % 8 || q->stride[1] % 8 || out->stride[0] % 8 || out->stride[1] % 8)
     return fail(PA_ERR_INVALID_ARG, "q/out rows must be contiguous and 16-byte aligned");
