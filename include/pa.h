@@ -229,9 +229,11 @@ int pa_prefill(pa_tensor* out, const pa_tensor* q, const pa_tensor* k_cache, con
                int32_t max_query_len, float scale, int32_t num_kv_heads, int32_t kernel, void* stream);
 
 /* Partition size pa_decode uses when opts->partition_tokens == 0 and a workspace is given
- * (0 = no split: the batch's B * Hkv (sequence, KV head) units already fill the GPU and every
- * context fits one CTA, <= 2048 tokens). Otherwise the largest of 2048, 1024, 512 that still gives
- * about four CTAs per SM, else 256. Host only. */
+ * (0 = no split: the batch's B * Hkv (sequence, KV head) units already fill the GPU, B * Hkv >= 592,
+ * and every context fits one CTA, <= 2048 tokens). Otherwise the largest of 2048, 1024 and 512
+ * shorter than max_context_len that still gives about four CTAs per SM,
+ * B * Hkv * ceil(max_context_len / size) >= 592; else 256, or 0 when max_context_len <= 256.
+ * Host only. */
 int32_t pa_decode_partition_tokens(int32_t num_seqs, int32_t num_kv_heads, int32_t max_context_len);
 
 /* Workspace bytes pa_decode needs for these sizes (0 when no split happens; SIZE_MAX when the size

@@ -312,3 +312,25 @@ def test_batch_incref_and_free_are_all_or_nothing(n, pre, batch, free):
     # The free lists agree in content and order: n allocations drain them identically.
     got = [lib.pa_block_alloc(a._h) for _ in range(a.num_free)]
     assert got == [want.alloc() for _ in range(want.num_free)]
+
+
+def _partition_rule(B, Hkv, ctx):
+    """The partition rule as pa.h states it, restated for the test."""
+    units = B * Hkv
+    if ctx <= 2048 and units >= 592:
+        return 0
+    for size in (2048, 1024, 512):
+        if ctx > size and units * -(-ctx // size) >= 592:
+            return size
+    return 256 if ctx > 256 else 0
+
+
+@settings(max_examples=400, deadline=None)
+@given(B=st.integers(1, 300), Hkv=st.sampled_from([1, 2, 4, 8, 32]), ctx=st.integers(1, 200000),
+       G=st.sampled_from([1, 4, 8]), D=st.sampled_from([64, 128]))
+def test_partition_rule_and_workspace_size(B, Hkv, ctx, G, D):
+    pt = pa.pa_decode_partition_tokens(B, Hkv, ctx)
+    assert pt == _partition_rule(B, Hkv, ctx)
+    P = -(-ctx // pt) if pt else 1
+    want = 0 if P <= 1 else -(-(B * Hkv * G * P * D * 4) // 256) * 256 + -(-(B * Hkv * G * P * 2 * 4) // 256) * 256
+    assert pa.pa_decode_workspace_bytes(B, Hkv * G, Hkv, D, ctx, 0) == want
