@@ -19,6 +19,9 @@ Readings taken where the pages are silent:
 * a block shared by several sequences carries a reference count, and returns to
   the free list when the count falls to zero;
 * unused block-table entries hold -1;
+* with a shared prefix, each prefix block is allocated once, by the first
+  sequence that reaches it, and every later sequence reaching it takes a
+  reference to it;
 * copy-on-write (前世今生 §3.2 names it for shared blocks): before a sequence writes into a block
   that other sequences also reference, it takes a fresh block, copies the page into it and moves
   its reference there.
