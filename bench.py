@@ -107,11 +107,22 @@ class ClockSampler:
             import pynvml
             pynvml.nvmlInit()
             self._nv = pynvml
-            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self._h, self.matched_by = self.nvml_handle(pynvml, device_index)
             self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
             self._ok = True
         except Exception as e:  # no NVML: report that instead of clocks
             self.error = f"{type(e).__name__}: {e}"
+
+    @staticmethod
+    def nvml_handle(nv, device_index: int):
+        """NVML handle of the GPU torch calls cuda:device_index. NVML numbers every GPU of the machine
+        while CUDA numbers only the visible ones (CUDA_VISIBLE_DEVICES), so match by UUID; fall back
+        to the index when the UUID is not available."""
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            return nv.nvmlDeviceGetHandleByUUID("GPU-" + uuid), "uuid"
+        except Exception:
+            return nv.nvmlDeviceGetHandleByIndex(device_index), "index"
 
     def _run(self):
         while not self._stop.is_set():
@@ -142,7 +153,7 @@ class ClockSampler:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "error": self.error}
         names = [n for n, bit in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
         return {"sm_mhz": statistics.median(self.samples) if self.samples else None, "sm_max_mhz": self.max_mhz,
-                "reasons": names, "samples": len(self.samples)}
+                "reasons": names, "samples": len(self.samples), "nvml_device_matched_by": self.matched_by}
 
 
 # ---------------------------------------------------------------------------------------------

@@ -42,3 +42,33 @@ def test_recorded_traffic_needs_a_matching_hash(tmp_path, monkeypatch):
     (tmp_path / "repo" / "profiles" / "decode_traffic.json").write_text(json.dumps(rec))
     assert bench.ncu_traffic("w") is None
     assert bench.ncu_traffic("missing") is None
+
+
+class _FakeNvml:
+    """Stands in for pynvml: two GPUs, the visible one is the second of the machine."""
+    NVML_CLOCK_SM = 0
+
+    def __init__(self):
+        self.calls = []
+
+    def nvmlDeviceGetHandleByUUID(self, uuid):
+        self.calls.append(("uuid", uuid))
+        return {"GPU-bbbb": "gpu1"}[uuid]
+
+    def nvmlDeviceGetHandleByIndex(self, i):
+        self.calls.append(("index", i))
+        return ["gpu0", "gpu1"][i]
+
+
+def test_clock_sampler_reads_the_timed_gpu_by_uuid(monkeypatch):
+    """cuda:0 is the machine's second GPU when CUDA_VISIBLE_DEVICES hides the first: NVML index 0
+    would sample the wrong GPU, its UUID does not."""
+    import types
+    nv = _FakeNvml()
+    monkeypatch.setattr(bench.torch.cuda, "get_device_properties", lambda i: types.SimpleNamespace(uuid="bbbb"))
+    assert bench.ClockSampler.nvml_handle(nv, 0) == ("gpu1", "uuid")
+
+    def no_props(i):
+        raise RuntimeError("no CUDA")
+    monkeypatch.setattr(bench.torch.cuda, "get_device_properties", no_props)
+    assert bench.ClockSampler.nvml_handle(nv, 0) == ("gpu0", "index")
