@@ -23,6 +23,17 @@
 //    O^T[D x 8g] += V^T[D x 16] . P^T. K/V fragments come from ldmatrix (V transposed by
 //    ldmatrix.trans); e4m3 pages are widened to f16 in registers (exact).
 //  * CUDA-core (kernel 0): float32 FMA dot products and axpys, kept for comparison (opts.kernel 0).
+//
+// Two modes ride on the same kernel:
+//  * pa_decode_step: the CTA of a sequence's last partition writes the new token's K/V row into
+//    its slot (the Cache Engine write) and fences it for the asynchronous proxy before any copy of
+//    that block's page is issued; the copies of its other first pages go out before the write, so
+//    the write overlaps them.
+//  * pa_decode_cascade (suffix grid): the CTAs cover tokens [shared prefix, context) and, while
+//    the prefix kernel before them on the stream still runs, wait for it only before reading its
+//    partials, which they fold into their own merge (or leave to reduce_kernel when the suffix
+//    itself is split). The CTA of KV head 0, partition 0 of each sequence checks that its table
+//    maps the prefix to sequence 0's blocks.
 #include <cfloat>
 #include <utility>
 
