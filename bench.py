@@ -733,6 +733,10 @@ def run_kv_utilization(args, rank):
 def main():
     args = parse()
     rank, world, local_rank = dist_env()
+    if args.gpus != world and rank == 0:
+        # Ranks come from the launcher (torch.distributed.run); the line reports the ranks that ran.
+        print(f"bench.py: --gpus {args.gpus} but {world} rank(s) launched; measuring {world} "
+              f"(launch N ranks with python -m torch.distributed.run --nproc-per-node N)", file=sys.stderr)
     if args.op == "kv_utilization":
         run_kv_utilization(args, rank)
         return 0
