@@ -368,7 +368,7 @@ class BlockAllocator:
         self._order = order  # keep alive during create
         h = _lib.pa_allocator_create(int(num_blocks), _i32_ptr(order) if order is not None else None)
         if not h:
-            raise ValueError("pa_allocator_create failed (bad num_blocks or initial_order)")
+            raise ValueError(f"pa_allocator_create: {pa_last_error()}")
         self._h = ctypes.c_void_p(h)
         self._destroy = _lib.pa_allocator_destroy  # still reachable during interpreter shutdown
 

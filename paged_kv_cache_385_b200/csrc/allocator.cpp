@@ -16,6 +16,9 @@
 #include <vector>
 
 #include "../../include/pa.h"
+#include "internal.h"
+
+using pa::set_last_error;
 
 struct pa_allocator {
   std::vector<int32_t> stack;  // free ids; top = back
@@ -32,7 +35,7 @@ int check_batch(const pa_allocator* a, int32_t n, const int32_t* blocks, int del
   try {
     ids.assign(blocks, blocks + n);
   } catch (...) {
-    return PA_ERR_INVALID_ARG;
+    return set_last_error(PA_ERR_INVALID_ARG, "out of host memory");
   }
   std::sort(ids.begin(), ids.end());
   const int32_t num_blocks = static_cast<int32_t>(a->ref.size());
@@ -41,9 +44,13 @@ int check_batch(const pa_allocator* a, int32_t n, const int32_t* blocks, int del
     size_t j = i;
     while (j < ids.size() && ids[j] == b) ++j;
     const int64_t times = static_cast<int64_t>(j - i);
-    if (b < 0 || b >= num_blocks || a->ref[b] == 0) return PA_ERR_BAD_BLOCK;
-    if (delta < 0 && times > a->ref[b]) return PA_ERR_BAD_BLOCK;
-    if (delta > 0 && a->ref[b] + times > INT32_MAX) return PA_ERR_INVALID_ARG;
+    if (b < 0 || b >= num_blocks || a->ref[b] == 0)
+      return set_last_error(PA_ERR_BAD_BLOCK, "block %d is not allocated (pool of %d)", b, num_blocks);
+    if (delta < 0 && times > a->ref[b])
+      return set_last_error(PA_ERR_BAD_BLOCK, "block %d listed %lld times but referenced %d times", b,
+                            static_cast<long long>(times), a->ref[b]);
+    if (delta > 0 && a->ref[b] + times > INT32_MAX)
+      return set_last_error(PA_ERR_INVALID_ARG, "reference count of block %d would overflow", b);
     i = j;
   }
   return PA_OK;
@@ -54,14 +61,21 @@ int check_batch(const pa_allocator* a, int32_t n, const int32_t* blocks, int del
 extern "C" {
 
 pa_allocator* pa_allocator_create(int32_t num_blocks, const int32_t* initial_order) {
-  if (num_blocks <= 0) return nullptr;
+  if (num_blocks <= 0) {
+    set_last_error(PA_ERR_INVALID_ARG, "num_blocks must be > 0 (got %d)", num_blocks);
+    return nullptr;
+  }
   pa_allocator* a = new (std::nothrow) pa_allocator;
-  if (!a) return nullptr;
+  if (!a) {
+    set_last_error(PA_ERR_INVALID_ARG, "out of host memory");
+    return nullptr;
+  }
   try {
     a->ref.assign(static_cast<size_t>(num_blocks), 0);
     a->stack.resize(static_cast<size_t>(num_blocks));
   } catch (...) {
     delete a;
+    set_last_error(PA_ERR_INVALID_ARG, "out of host memory for %d blocks", num_blocks);
     return nullptr;
   }
   if (initial_order) {
@@ -71,6 +85,8 @@ pa_allocator* pa_allocator_create(int32_t num_blocks, const int32_t* initial_ord
       const int32_t b = initial_order[i];
       if (b < 0 || b >= num_blocks || seen[b]) {
         delete a;
+        set_last_error(PA_ERR_INVALID_ARG, "initial_order is not a permutation of [0, %d): entry %d is %d",
+                       num_blocks, i, b);
         return nullptr;
       }
       seen[b] = 1;
@@ -85,8 +101,8 @@ pa_allocator* pa_allocator_create(int32_t num_blocks, const int32_t* initial_ord
 void pa_allocator_destroy(pa_allocator* a) { delete a; }
 
 int32_t pa_block_alloc(pa_allocator* a) {
-  if (!a) return PA_ERR_INVALID_ARG;
-  if (a->stack.empty()) return PA_ERR_EXHAUSTED;
+  if (!a) return set_last_error(PA_ERR_INVALID_ARG, "allocator is NULL");
+  if (a->stack.empty()) return set_last_error(PA_ERR_EXHAUSTED, "all %zu blocks are in use", a->ref.size());
   const int32_t b = a->stack.back();
   a->stack.pop_back();
   a->ref[b] = 1;
@@ -94,28 +110,32 @@ int32_t pa_block_alloc(pa_allocator* a) {
 }
 
 int pa_block_incref(pa_allocator* a, int32_t b) {
-  if (!a) return PA_ERR_INVALID_ARG;
-  if (b < 0 || b >= static_cast<int32_t>(a->ref.size()) || a->ref[b] == 0) return PA_ERR_BAD_BLOCK;
-  if (a->ref[b] == INT32_MAX) return PA_ERR_INVALID_ARG;
+  if (!a) return set_last_error(PA_ERR_INVALID_ARG, "allocator is NULL");
+  if (b < 0 || b >= static_cast<int32_t>(a->ref.size()) || a->ref[b] == 0)
+    return set_last_error(PA_ERR_BAD_BLOCK, "block %d is not allocated", b);
+  if (a->ref[b] == INT32_MAX) return set_last_error(PA_ERR_INVALID_ARG, "reference count of block %d would overflow", b);
   ++a->ref[b];
   return PA_OK;
 }
 
 int pa_block_free(pa_allocator* a, int32_t b) {
-  if (!a) return PA_ERR_INVALID_ARG;
-  if (b < 0 || b >= static_cast<int32_t>(a->ref.size()) || a->ref[b] == 0) return PA_ERR_BAD_BLOCK;
+  if (!a) return set_last_error(PA_ERR_INVALID_ARG, "allocator is NULL");
+  if (b < 0 || b >= static_cast<int32_t>(a->ref.size()) || a->ref[b] == 0)
+    return set_last_error(PA_ERR_BAD_BLOCK, "block %d is not allocated", b);
   if (--a->ref[b] == 0) a->stack.push_back(b);
   return PA_OK;
 }
 
 int pa_block_cow(pa_allocator* a, int32_t b, int32_t* out_block) {
-  if (!a || !out_block) return PA_ERR_INVALID_ARG;
-  if (b < 0 || b >= static_cast<int32_t>(a->ref.size()) || a->ref[b] == 0) return PA_ERR_BAD_BLOCK;
+  if (!a || !out_block) return set_last_error(PA_ERR_INVALID_ARG, "allocator or out_block is NULL");
+  if (b < 0 || b >= static_cast<int32_t>(a->ref.size()) || a->ref[b] == 0)
+    return set_last_error(PA_ERR_BAD_BLOCK, "block %d is not allocated", b);
   if (a->ref[b] == 1) {  // sole owner: write in place
     *out_block = b;
     return 0;
   }
-  if (a->stack.empty()) return PA_ERR_EXHAUSTED;
+  if (a->stack.empty())
+    return set_last_error(PA_ERR_EXHAUSTED, "block %d is shared and no block is free for its copy", b);
   const int32_t nb = pa_block_alloc(a);
   --a->ref[b];
   *out_block = nb;
@@ -123,8 +143,9 @@ int pa_block_cow(pa_allocator* a, int32_t b, int32_t* out_block) {
 }
 
 int32_t pa_block_refcount(const pa_allocator* a, int32_t b) {
-  if (!a) return PA_ERR_INVALID_ARG;
-  if (b < 0 || b >= static_cast<int32_t>(a->ref.size())) return PA_ERR_BAD_BLOCK;
+  if (!a) return set_last_error(PA_ERR_INVALID_ARG, "allocator is NULL");
+  if (b < 0 || b >= static_cast<int32_t>(a->ref.size()))
+    return set_last_error(PA_ERR_BAD_BLOCK, "block %d is outside the pool of %zu", b, a->ref.size());
   return a->ref[b];
 }
 
@@ -133,8 +154,9 @@ int32_t pa_allocator_num_free(const pa_allocator* a) { return a ? static_cast<in
 int32_t pa_allocator_num_blocks(const pa_allocator* a) { return a ? static_cast<int32_t>(a->ref.size()) : PA_ERR_INVALID_ARG; }
 
 int pa_blocks_alloc_n(pa_allocator* a, int32_t n, int32_t* out) {
-  if (!a || n < 0 || (n > 0 && !out)) return PA_ERR_INVALID_ARG;
-  if (static_cast<size_t>(n) > a->stack.size()) return PA_ERR_EXHAUSTED;
+  if (!a || n < 0 || (n > 0 && !out)) return set_last_error(PA_ERR_INVALID_ARG, "NULL allocator or output, or n < 0");
+  if (static_cast<size_t>(n) > a->stack.size())
+    return set_last_error(PA_ERR_EXHAUSTED, "%d blocks asked for, %zu free", n, a->stack.size());
   for (int32_t i = 0; i < n; ++i) out[i] = pa_block_alloc(a);
   return PA_OK;
 }
@@ -142,14 +164,14 @@ int pa_blocks_alloc_n(pa_allocator* a, int32_t n, int32_t* out) {
 // Both batch calls are all-or-nothing: the whole list is checked first, then applied in list order
 // (so blocks whose last reference goes are pushed in that order, as n single frees would).
 int pa_blocks_incref_n(pa_allocator* a, int32_t n, const int32_t* blocks) {
-  if (!a || n < 0 || (n > 0 && !blocks)) return PA_ERR_INVALID_ARG;
+  if (!a || n < 0 || (n > 0 && !blocks)) return set_last_error(PA_ERR_INVALID_ARG, "NULL allocator or blocks, or n < 0");
   if (const int r = check_batch(a, n, blocks, +1)) return r;
   for (int32_t i = 0; i < n; ++i) ++a->ref[blocks[i]];
   return PA_OK;
 }
 
 int pa_blocks_free_n(pa_allocator* a, int32_t n, const int32_t* blocks) {
-  if (!a || n < 0 || (n > 0 && !blocks)) return PA_ERR_INVALID_ARG;
+  if (!a || n < 0 || (n > 0 && !blocks)) return set_last_error(PA_ERR_INVALID_ARG, "NULL allocator or blocks, or n < 0");
   if (const int r = check_batch(a, n, blocks, -1)) return r;
   for (int32_t i = 0; i < n; ++i)
     if (--a->ref[blocks[i]] == 0) a->stack.push_back(blocks[i]);
@@ -160,14 +182,20 @@ int pa_slots_for_positions(const int32_t* bt, int64_t row_stride, int32_t num_se
                            const int32_t* token_seq, const int32_t* token_pos, int64_t num_tokens, int64_t* out) {
   if (num_tokens < 0 || (num_tokens > 0 && (!bt || !token_seq || !token_pos || !out)) || num_seqs < 0 ||
       max_blocks < 0 || row_stride < max_blocks)
-    return PA_ERR_INVALID_ARG;
+    return set_last_error(PA_ERR_INVALID_ARG, "NULL pointer, negative count or row_stride < max_blocks");
   for (int64_t i = 0; i < num_tokens; ++i) {
     const int32_t s = token_seq[i], pos = token_pos[i];
-    if (s < 0 || s >= num_seqs || pos < 0) return PA_ERR_INVALID_ARG;
+    if (s < 0 || s >= num_seqs || pos < 0)
+      return set_last_error(PA_ERR_INVALID_ARG, "token %lld: sequence %d / position %d out of range",
+                            static_cast<long long>(i), s, pos);
     const int32_t j = pos / PA_BLOCK_SIZE;
-    if (j >= max_blocks) return PA_ERR_INVALID_ARG;
+    if (j >= max_blocks)
+      return set_last_error(PA_ERR_INVALID_ARG, "token %lld: position %d is past the table's %d blocks",
+                            static_cast<long long>(i), pos, max_blocks);
     const int32_t b = bt[static_cast<int64_t>(s) * row_stride + j];
-    if (b < 0) return PA_ERR_INVALID_ARG;
+    if (b < 0)
+      return set_last_error(PA_ERR_INVALID_ARG, "token %lld: table entry %d of sequence %d is %d",
+                            static_cast<long long>(i), j, s, b);
     out[i] = static_cast<int64_t>(b) * PA_BLOCK_SIZE + pos % PA_BLOCK_SIZE;
   }
   return PA_OK;

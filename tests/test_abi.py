@@ -334,3 +334,22 @@ def test_partition_rule_and_workspace_size(B, Hkv, ctx, G, D):
     P = -(-ctx // pt) if pt else 1
     want = 0 if P <= 1 else -(-(B * Hkv * G * P * D * 4) // 256) * 256 + -(-(B * Hkv * G * P * 2 * 4) // 256) * 256
     assert pa.pa_decode_workspace_bytes(B, Hkv * G, Hkv, D, ctx, 0) == want
+
+
+def test_allocator_errors_carry_a_reason():
+    lib = pa.lib()
+    assert not lib.pa_allocator_create(0, None)
+    assert "num_blocks" in pa.pa_last_error()
+    bad = torch.tensor([0, 2, 2], dtype=torch.int32)
+    assert not lib.pa_allocator_create(3, pa._i32_ptr(bad))
+    assert "permutation" in pa.pa_last_error()
+    a = pa.BlockAllocator(2)
+    a.alloc_n(2)
+    with pytest.raises(pa.PagedAttentionError, match="2 blocks are in use"):
+        a.alloc()
+    with pytest.raises(pa.PagedAttentionError, match="block 7 is not allocated"):
+        a.incref(7)
+    with pytest.raises(pa.PagedAttentionError, match="listed 2 times but referenced 1"):
+        a.free_n(torch.tensor([1, 1], dtype=torch.int32))
+    with pytest.raises(pa.PagedAttentionError, match="past the table"):
+        pa.pa_slots_for_positions(torch.tensor([[0, 1]], dtype=torch.int32), [0], [40])
