@@ -353,3 +353,11 @@ def test_allocator_errors_carry_a_reason():
         a.free_n(torch.tensor([1, 1], dtype=torch.int32))
     with pytest.raises(pa.PagedAttentionError, match="past the table"):
         pa.pa_slots_for_positions(torch.tensor([[0, 1]], dtype=torch.int32), [0], [40])
+
+
+def test_binding_declares_every_entry_point():
+    """The ctypes binding gives every function of the header its argument and result types (a call
+    through an undeclared signature would pass Python ints as C ints and truncate pointers)."""
+    lib = pa.lib()
+    undeclared = [n for n in declared_functions() if getattr(lib, n).argtypes is None]
+    assert not undeclared, undeclared
