@@ -361,3 +361,18 @@ def test_binding_declares_every_entry_point():
     lib = pa.lib()
     undeclared = [n for n in declared_functions() if getattr(lib, n).argtypes is None]
     assert not undeclared, undeclared
+
+
+def test_binding_signatures_match_the_header_arity():
+    """Each ctypes signature has as many arguments as the header's prototype."""
+    protos = {}
+    for hdr in os.listdir(os.path.join(ROOT, "include")):
+        if hdr.endswith(".h"):
+            text = re.sub(r"/\*.*?\*/", "", open(os.path.join(ROOT, "include", hdr)).read(), flags=re.S)
+            for name, params in re.findall(r"\b(pa_[a-z0-9_]+)\s*\(([^;{}]*?)\)\s*;", text):
+                p = " ".join(params.split())
+                protos[name] = 0 if p in ("", "void") else p.count(",") + 1
+    lib = pa.lib()
+    assert set(protos) == set(declared_functions())
+    wrong = {n: (k, len(getattr(lib, n).argtypes)) for n, k in protos.items() if len(getattr(lib, n).argtypes) != k}
+    assert not wrong, wrong
