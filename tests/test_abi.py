@@ -376,3 +376,29 @@ def test_binding_signatures_match_the_header_arity():
     assert set(protos) == set(declared_functions())
     wrong = {n: (k, len(getattr(lib, n).argtypes)) for n, k in protos.items() if len(getattr(lib, n).argtypes) != k}
     assert not wrong, wrong
+
+
+def test_struct_layouts_match_the_header(tmp_path):
+    """The ctypes mirrors of pa_tensor and pa_decode_opts have the C structs' sizes and field offsets
+    (compiled from include/pa.h with the host C compiler)."""
+    import shutil
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no host C compiler")
+    fields = {"pa_tensor": [f[0] for f in pa.PaTensor._fields_],
+              "pa_decode_opts": [f[0] for f in pa.PaDecodeOpts._fields_]}
+    lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "pa.h"', "int main(void) {"]
+    for st_, names in fields.items():
+        lines.append(f'  printf("{st_} size %zu\\n", sizeof({st_}));')
+        lines += [f'  printf("{st_} {n} %zu\\n", offsetof({st_}, {n}));' for n in names]
+    lines += ["  return 0;", "}"]
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines))
+    exe = tmp_path / "layout"
+    subprocess.run([cc, "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
+    got = dict(ln.rsplit(" ", 1) for ln in subprocess.run([str(exe)], capture_output=True, text=True,
+                                                          check=True).stdout.splitlines())
+    for st_, cls in (("pa_tensor", pa.PaTensor), ("pa_decode_opts", pa.PaDecodeOpts)):
+        assert int(got[f"{st_} size"]) == ctypes.sizeof(cls)
+        for n in fields[st_]:
+            assert int(got[f"{st_} {n}"]) == getattr(cls, n).offset, (st_, n)
