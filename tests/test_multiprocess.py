@@ -32,7 +32,7 @@ def _worker(rank, world, port, results):
 
 def test_two_replicas_take_the_slowest_rank():
     world = 2
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:  # no fork of this (multi-threaded) process
         results = m.dict()
         mp.spawn(_worker, args=(world, _free_port(), results), nprocs=world, join=True)
         res = dict(results)
