@@ -280,6 +280,14 @@ const char* pa_last_error(void);
  * into *bits and, if clear != 0, reset it to 0. Not for hot paths. */
 int pa_read_device_error(uint32_t* bits, int clear);
 
+/* Host-side fault injection for testing a caller's error handling: the next `count` calls of
+ * pa_reshape_and_cache, pa_decode, pa_decode_step, pa_decode_cascade, pa_decode_no_alloc,
+ * pa_prefill and pa_copy_blocks that reach their first device call (every argument check passed
+ * and there is work to enqueue) return PA_ERR_CUDA without any device work, as a call whose launch failed does (nothing is enqueued, pa_last_error says it was
+ * injected). count 0 disarms. Process-wide; thread-safe. Nothing reaches the GPU: no device-side
+ * fault is ever made. Returns PA_OK, or PA_ERR_INVALID_ARG for count < 0. */
+int pa_debug_fail_next_launches(int32_t count);
+
 /* Library version, "major.minor.patch". */
 const char* pa_version(void);
 

@@ -89,6 +89,7 @@ def _load() -> ctypes.CDLL:
         "pa_last_error": (ctypes.c_char_p, []),
         "pa_read_device_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), ctypes.c_int]),
         "pa_version": (ctypes.c_char_p, []),
+        "pa_debug_fail_next_launches": (ctypes.c_int, [I32]),
         "pa_selftest_bounded_wait": (ctypes.c_int, [I32, ctypes.c_void_p, VP]),
         "pa_allocator_create": (VP, [I32, i32p]),
         "pa_allocator_destroy": (None, [VP]),
@@ -337,6 +338,12 @@ def pa_last_error() -> str:
 
 def pa_version() -> str:
     return _lib.pa_version().decode()
+
+
+def pa_debug_fail_next_launches(count: int) -> None:
+    """Host-side fault injection: the next ``count`` calls that pass their argument checks raise
+    PagedAttentionError(PA_ERR_CUDA) without device work, as a failed launch does (see include/pa.h)."""
+    _check(_lib.pa_debug_fail_next_launches(int(count)), "pa_debug_fail_next_launches")
 
 
 def _i32_ptr(t: torch.Tensor):

@@ -146,6 +146,17 @@ int encode_q_map(CUtensorMap* map, const pa_tensor* q, int group) {
   return PA_OK;
 }
 
+// Host-side fault injection (pa_debug_fail_next_launches): calls left that fail as a launch would.
+std::atomic<int32_t> g_injected_failures{0};
+
+// True (and one fewer left) when this call is to fail as if its launch had failed.
+bool take_injected_failure() {
+  int32_t n = g_injected_failures.load(std::memory_order_relaxed);
+  while (n > 0 && !g_injected_failures.compare_exchange_weak(n, n - 1, std::memory_order_relaxed)) {
+  }
+  return n > 0;
+}
+
 // The device address of the library's error word, looked up once per device. Threads may race on
 // the first lookup; they all store the same address, and the slots are atomics so that is well defined.
 uint32_t* library_error_word() {
@@ -249,6 +260,12 @@ size_t pa_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t 
   return workspace_layout(num_seqs, num_q_heads, head_dim, P, nullptr);
 }
 
+int pa_debug_fail_next_launches(int32_t count) {
+  if (count < 0) return fail(PA_ERR_INVALID_ARG, "count must be >= 0");
+  g_injected_failures.store(count, std::memory_order_relaxed);
+  return ok();
+}
+
 int pa_read_device_error(uint32_t* bits, int clear) {
   if (!bits) return fail(PA_ERR_INVALID_ARG, "bits is NULL");
   cudaError_t e = pa::read_and_clear_error_word(bits, clear);
@@ -320,6 +337,7 @@ int pa_reshape_and_cache(const pa_tensor* key, const pa_tensor* value, const pa_
     p.k_inv_scale = one / k_scale;
     p.v_inv_scale = one / v_scale;
   }
+  if (take_injected_failure()) return fail(PA_ERR_CUDA, "injected launch failure (pa_debug_fail_next_launches)");
   p.err = library_error_word();
   if (!p.err) return fail(PA_ERR_CUDA, "no device error word (no current CUDA device?)");
   const pa::KvType kv = cd == PA_E4M3 ? pa::KvType::E4M3 : (cd == PA_BF16 ? pa::KvType::BF16 : pa::KvType::F16);
@@ -532,6 +550,7 @@ static int decode_impl(pa_tensor* out, const pa_tensor* q, const pa_tensor* k_ca
   }
 
   // Every argument check is above: the device calls start here.
+  if (take_injected_failure()) return fail(PA_ERR_CUDA, "injected launch failure (pa_debug_fail_next_launches)");
   p.err = opts.error_word ? reinterpret_cast<uint32_t*>(opts.error_word) : library_error_word();
   if (!p.err) return fail(PA_ERR_CUDA, "no device error word (no current CUDA device?)");
   if (builtin && ws_parts > 1) {
@@ -614,6 +633,7 @@ int pa_copy_blocks(pa_tensor* k_cache, pa_tensor* v_cache, const pa_tensor* bloc
   p.num_pairs = N;
   p.block_bytes = block_bytes;
   p.num_blocks = k_cache->shape[0];
+  if (take_injected_failure()) return fail(PA_ERR_CUDA, "injected launch failure (pa_debug_fail_next_launches)");
   p.err = library_error_word();
   if (!p.err) return fail(PA_ERR_CUDA, "no device error word (no current CUDA device?)");
   cudaError_t e = pa::launch_copy_blocks(p, static_cast<cudaStream_t>(stream));
@@ -736,6 +756,7 @@ int pa_prefill(pa_tensor* out, const pa_tensor* q, const pa_tensor* k_cache, con
   p.group = static_cast<int32_t>(Hq / num_kv_heads);
   p.max_blocks = static_cast<int32_t>(std::min<int64_t>(block_tables->shape[1], 0x7fffffff / 16));
   p.score_scale_log2 = scale * 1.4426950408889634f;
+  if (take_injected_failure()) return fail(PA_ERR_CUDA, "injected launch failure (pa_debug_fail_next_launches)");
   p.err = library_error_word();
   if (!p.err) return fail(PA_ERR_CUDA, "no device error word (no current CUDA device?)");
   CUtensorMap km, vm;

@@ -1,0 +1,88 @@
+"""Host-side fault injection (pa_debug_fail_next_launches): calls fail as a failed launch does,
+with no device work, and argument errors still come first.
+
+The descriptors point at host memory, so this runs only where no CUDA device is present (there the
+calls that are not injected stop at the first CUDA call; on a GPU they would launch kernels on host
+pointers). The hook itself never reaches a device.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import paged_kv_cache_385_b200 as pa
+
+pytestmark = pytest.mark.skipif(torch.cuda.is_available(),
+                                reason="host-pointer descriptors must never reach a GPU launch")
+
+
+def _aligned(shape, dtype, align=256):
+    n = int(np.prod(shape)) * torch.tensor([], dtype=dtype).element_size()
+    raw = torch.zeros(n + align, dtype=torch.uint8)
+    off = (-raw.data_ptr()) % align
+    return raw[off:off + n].view(dtype).view(*shape)
+
+
+@pytest.fixture
+def decode_args():
+    B, Hq, Hkv, D, NB = 2, 8, 2, 128, 16
+    q = _aligned((B, Hq, D), torch.bfloat16)
+    kc = _aligned((NB, Hkv, 16, D), torch.bfloat16)
+    bt = torch.zeros(B, 4, dtype=torch.int32)
+    lens = torch.full((B,), 40, dtype=torch.int32)
+    ts = [pa.as_pa_tensor(t, n, device=False) for t, n in ((q, "out"), (q, "q"), (kc, "k"), (kc, "v"), (bt, "bt"),
+                                                            (lens, "lens"))]
+    keep = (q, kc, bt, lens)
+
+    def call(hkv=Hkv):
+        return pa.lib().pa_decode(*[ctypes.byref(t) for t in ts], 0.088, hkv, None, None)
+    call.keep = keep
+    return call
+
+
+def test_injected_failures_are_counted_and_host_only(decode_args):
+    try:
+        pa.pa_debug_fail_next_launches(2)
+        assert decode_args() == pa.PA_ERR_CUDA and "injected" in pa.pa_last_error()
+        # An argument error is reported as such and does not use up an injected failure.
+        assert decode_args(hkv=3) == pa.PA_ERR_INVALID_ARG
+        assert decode_args() == pa.PA_ERR_CUDA and "injected" in pa.pa_last_error()
+        # Both used: the next call goes on to the device (none here: a real CUDA error).
+        assert decode_args() == pa.PA_ERR_CUDA and "injected" not in pa.pa_last_error()
+    finally:
+        pa.pa_debug_fail_next_launches(0)
+
+
+def test_every_enqueuing_entry_point_takes_the_hook():
+    T, Hkv, D, NB = 3, 2, 64, 8
+    key = _aligned((T, Hkv, D), torch.float16)
+    kc = _aligned((NB, Hkv, 16, D), torch.float16)
+    slots = torch.zeros(T, dtype=torch.int64)
+    mapping = torch.tensor([[0, 1]], dtype=torch.int64)
+    q = _aligned((T, Hkv, D), torch.float16)
+    bt = torch.zeros(1, 1, dtype=torch.int32)
+    qs = torch.tensor([0, T], dtype=torch.int32)
+    lens = torch.tensor([T], dtype=torch.int32)
+    P = lambda t, n: ctypes.byref(pa.as_pa_tensor(t, n, device=False))  # noqa: E731
+    lib = pa.lib()
+    calls = {
+        "pa_reshape_and_cache": lambda: lib.pa_reshape_and_cache(P(key, "k"), P(key, "v"), P(slots, "s"), P(kc, "kc"),
+                                                                 P(kc, "vc"), 1.0, 1.0, None),
+        "pa_copy_blocks": lambda: lib.pa_copy_blocks(P(kc, "kc"), P(kc, "vc"), P(mapping, "m"), None),
+        "pa_prefill": lambda: lib.pa_prefill(P(q, "o"), P(q, "q"), P(kc, "kc"), P(kc, "vc"), P(bt, "bt"), P(qs, "qs"),
+                                             P(lens, "l"), T, 0.125, Hkv, -1, None),
+    }
+    try:
+        for name, call in calls.items():
+            pa.pa_debug_fail_next_launches(1)
+            assert call() == pa.PA_ERR_CUDA, name
+            assert "injected" in pa.pa_last_error(), name
+    finally:
+        pa.pa_debug_fail_next_launches(0)
+
+
+def test_negative_count_is_refused():
+    with pytest.raises(pa.PagedAttentionError) as e:
+        pa.pa_debug_fail_next_launches(-1)
+    assert e.value.status == pa.PA_ERR_INVALID_ARG
