@@ -236,6 +236,23 @@ def test_decode_argument_errors_are_reported_before_device_work():
     assert "workspace" in pa.pa_last_error()
     small = _aligned_zeros((64,), torch.uint8)
     assert call(partition_tokens=256, workspace=small.data_ptr(), workspace_bytes=64) == pa.PA_ERR_WORKSPACE
+    kc3 = _aligned_zeros((NB, 3, 16, D), torch.bfloat16)
+    assert call(kcache=kc3, hkv=3) == pa.PA_ERR_INVALID_ARG  # 8 query heads over 3 KV heads
+    assert "multiple" in pa.pa_last_error()
+    # Misaligned pointers: q / out rows, the pool, the workspace.
+    for i, off in ((1, 2), (2, 64)):
+        ts = [pa.as_pa_tensor(t, n, device=False) for t, n in ((q, "out"), (q, "q"), (kc, "k"), (kc, "v"),
+                                                                (bt, "bt"), (lens, "lens"))]
+        ts[i].data += off
+        opts = pa.PaDecodeOpts()
+        lib.pa_decode_opts_init(ctypes.byref(opts))
+        assert lib.pa_decode(*[ctypes.byref(t) for t in ts], 0.088, Hkv, ctypes.byref(opts), None) == \
+            pa.PA_ERR_INVALID_ARG
+        assert "aligned" in pa.pa_last_error()
+    big = _aligned_zeros((1 << 20,), torch.uint8)
+    assert call(partition_tokens=256, workspace=big.data_ptr() + 8, workspace_bytes=(1 << 20) - 8) == \
+        pa.PA_ERR_INVALID_ARG
+    assert "aligned" in pa.pa_last_error()
 
 
 def test_shared_prefix_blocks_come_from_the_first_sequence_reaching_them():
