@@ -86,3 +86,58 @@ def test_negative_count_is_refused():
     with pytest.raises(pa.PagedAttentionError) as e:
         pa.pa_debug_fail_next_launches(-1)
     assert e.value.status == pa.PA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("cascade", [False, True])
+def test_queried_workspace_size_is_exactly_what_the_call_checks(cascade):
+    """A workspace of the size the query function reports passes the entry point's checks (the
+    armed failure is reached); one byte less is refused with PA_ERR_WORKSPACE when a split happens."""
+    rng = np.random.default_rng(5 + cascade)
+    lib = pa.lib()
+    checked = 0
+    for _ in range(150):
+        Hkv = int(rng.choice([1, 2, 8]))
+        G = int(rng.choice([1, 4, 8]))
+        B, D = int(rng.integers(1, 40)), int(rng.choice([64, 128]))
+        mb = int(rng.integers(1, 300))
+        max_ctx = int(rng.integers(1, mb * 16 + 1))
+        pt = int(rng.choice([0, 0, 16, 256, 512, 2048]))
+        prefix = 16 * int(rng.integers(1, mb + 1)) if cascade else 0
+        if cascade and D != 128:
+            D = 128
+        q = _aligned((B, Hkv * G, D), torch.bfloat16)
+        kc = _aligned((4, Hkv, 16, D), torch.bfloat16)
+        bt = torch.zeros(B, mb, dtype=torch.int32)
+        lens = torch.ones(B, dtype=torch.int32)
+        if cascade:
+            need = pa.pa_decode_cascade_workspace_bytes(B, Hkv * G, Hkv, D, max_ctx, prefix, pt)
+        else:
+            need = pa.pa_decode_workspace_bytes(B, Hkv * G, Hkv, D, max_ctx, pt)
+        ws = _aligned((max(need, 1),), torch.uint8)
+        ts = [pa.as_pa_tensor(t, n, device=False) for t, n in ((q, "out"), (q, "q"), (kc, "k"), (kc, "v"),
+                                                                (bt, "bt"), (lens, "lens"))]
+
+        def call(nbytes):
+            opts = pa.PaDecodeOpts()
+            lib.pa_decode_opts_init(ctypes.byref(opts))
+            opts.max_context_len, opts.partition_tokens = max_ctx, pt
+            if nbytes > 0:
+                opts.workspace, opts.workspace_bytes = ws.data_ptr(), nbytes
+            r = [ctypes.byref(t) for t in ts]
+            pa.pa_debug_fail_next_launches(1)
+            try:
+                if cascade:
+                    status = lib.pa_decode_cascade(r[0], r[1], None, None, None, r[2], r[3], r[4], r[5], prefix,
+                                                   0.1, Hkv, ctypes.byref(opts), None)
+                else:
+                    status = lib.pa_decode(*r, 0.1, Hkv, ctypes.byref(opts), None)
+                return status, pa.pa_last_error()  # read before the disarming call resets it
+            finally:
+                pa.pa_debug_fail_next_launches(0)
+
+        st_, msg = call(need)
+        assert st_ == pa.PA_ERR_CUDA and "injected" in msg, (msg, need)
+        if need > 0:
+            assert call(need - 1)[0] == pa.PA_ERR_WORKSPACE
+            checked += 1
+    assert checked > 20
