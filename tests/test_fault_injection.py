@@ -141,3 +141,34 @@ def test_queried_workspace_size_is_exactly_what_the_call_checks(cascade):
             assert call(need - 1)[0] == pa.PA_ERR_WORKSPACE
             checked += 1
     assert checked > 20
+
+
+def test_no_alloc_accepts_exactly_the_batches_its_array_holds():
+    rng = np.random.default_rng(11)
+    lib = pa.lib()
+    seen = set()
+    for _ in range(200):
+        Hkv, G = int(rng.choice([1, 8])), int(rng.choice([1, 8]))
+        B, D, mb = int(rng.integers(1, 64)), 128, int(rng.integers(1, 8192))
+        max_ctx, pt = int(rng.integers(1, mb * 16 + 1)), int(rng.choice([0, 256, 512]))
+        q = _aligned((B, Hkv * G, D), torch.bfloat16)
+        kc = _aligned((4, Hkv, 16, D), torch.bfloat16)
+        bt, lens = torch.zeros(B, mb, dtype=torch.int32), torch.ones(B, dtype=torch.int32)
+        ts = [pa.as_pa_tensor(t, n, device=False) for t, n in ((q, "out"), (q, "q"), (kc, "k"), (kc, "v"),
+                                                                (bt, "bt"), (lens, "lens"))]
+        opts = pa.PaDecodeOpts()
+        lib.pa_decode_opts_init(ctypes.byref(opts))
+        opts.max_context_len, opts.partition_tokens = max_ctx, pt
+        need = pa.pa_decode_workspace_bytes(B, Hkv * G, Hkv, D, max_ctx, pt)
+        pa.pa_debug_fail_next_launches(1)
+        try:
+            st_ = lib.pa_decode_no_alloc(*[ctypes.byref(t) for t in ts], 0.1, Hkv, ctypes.byref(opts), None)
+            msg = pa.pa_last_error()
+        finally:
+            pa.pa_debug_fail_next_launches(0)
+        if need <= pa.NO_ALLOC_SCRATCH_BYTES:
+            assert st_ == pa.PA_ERR_CUDA and "injected" in msg, (need, msg)
+        else:
+            assert st_ == pa.PA_ERR_WORKSPACE and "scratch" in msg, (need, msg)
+        seen.add(need <= pa.NO_ALLOC_SCRATCH_BYTES)
+    assert seen == {True, False}
