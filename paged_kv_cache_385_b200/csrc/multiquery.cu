@@ -190,11 +190,13 @@ __global__ void __launch_bounds__(PCfg<KV, D>::kThreads) mq_kernel(const __grid_
   const int t_tok = ((lane >> 4) << 3) | x7, t_co = (lane >> 3) & 1;          // K^T matrices
   const int a_tok = (((lane >> 3) & 1) << 3) | x7, a_co = lane >> 4;          // V^T matrices
 
+  int fail_at = 0;
   for (int i = 0; i < npages; ++i) {
     const int st = i % kPrefixStages;
     const bool got = mbar_wait_bounded(full0 + 8 * st, (i / kPrefixStages) & 1, deadline);
     if (!__all_sync(kFull, got)) {
       ok = false;
+      fail_at = i;
       if (lane == 0) atomicOr(p.err, 4u);
       break;
     }
@@ -282,7 +284,16 @@ __global__ void __launch_bounds__(PCfg<KV, D>::kThreads) mq_kernel(const __grid_
     if (lane == 0) mbar_arrive(empty0 + 8 * st);
   }
   if constexpr (kPrefill) pdl_launch_dependents();
-  if (!ok) return;
+  if (!ok) {
+    // Give the copies the producer may have issued for pages fail_at .. fail_at + stages - 1 a bounded
+    // chance to land before the CTA's shared memory goes. It cannot have issued any later page: that
+    // needs this warp's release of page fail_at's stage, and each earlier fill of those stages was
+    // consumed here, so the parity waits are exact.
+    const uint64_t drain_deadline = globaltimer_ns() + 100000000ull;
+    for (int k = fail_at; k < min(fail_at + kPrefixStages, npages); ++k)
+      mbar_wait_bounded(full0 + 8 * (k % kPrefixStages), (k / kPrefixStages) & 1, drain_deadline);
+    return;
+  }
 
   l_lo += __shfl_xor_sync(kFull, l_lo, 1);
   l_lo += __shfl_xor_sync(kFull, l_lo, 2);

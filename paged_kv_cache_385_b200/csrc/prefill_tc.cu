@@ -157,14 +157,15 @@ __global__ void __launch_bounds__(kThreads, 2)
   bool ok = true;
 
   // Producer of one stream (K by warp 4, V by warp 6): block j's 4 page ids, then its 8 tile copies
-  // into stage j % NS once that stage's previous block has been consumed.
-  auto produce = [&](const CUtensorMap* map, uint32_t off, int ns, int full0, int empty0) {
+  // into stage j % NS once that stage's previous block has been consumed. Returns the number of
+  // blocks whose copies it issued.
+  auto produce = [&](const CUtensorMap* map, uint32_t off, int ns, int full0, int empty0) -> int {
     const int oob_row = p.num_blocks * p.num_kv_heads * 16;  // a box starting here is all zero fill
     for (int j = 0; j < nkb; ++j) {
       const int st = j % ns;
       if (j >= ns && !mbar_wait_bounded(B(empty0 + st), ((j / ns) - 1) & 1, deadline)) {
         atomicOr(p.err, 4u);
-        return;
+        return j;
       }
       int ys[kKeys / 16];
 #pragma unroll
@@ -188,10 +189,12 @@ __global__ void __launch_bounds__(kThreads, 2)
       for (int i = 0; i < kKeys / 16; ++i)
         for (int u = 0; u < 2; ++u) tma_load_2d(dst + u * kHalfKV + i * 2048, map, B(full0 + st), u * 64, ys[i]);
     }
+    return nkb;
   };
+  int issued = 0;  // producer lanes: blocks of their stream whose copies they issued
 
   if (warp == 6) {
-    if (lane == 0) produce(&vmap, kVOff, kVStages, kVFull0, kVEmpty0);
+    if (lane == 0) issued = produce(&vmap, kVOff, kVStages, kVFull0, kVEmpty0);
   } else if (warp == 4) {
     // ---- producer -------------------------------------------------------------------------------
     if (lane == 0) {
@@ -200,7 +203,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       const int tok0 = q_row0 + tile * (kRows / G);
       tc05::tma_load_3d(base + kQOff, &qmap, B(kQFull), 0, hk * G, tok0);
       tc05::tma_load_3d(base + kQOff + kHalf, &qmap, B(kQFull), 64, hk * G, tok0);
-      produce(&kmap, kKOff, kKStages, kKFull0, kKEmpty0);
+      issued = produce(&kmap, kKOff, kKStages, kKFull0, kKEmpty0);
     }
   } else if (warp == 5) {
     // ---- QK issuer: S(j) = Q K(j)^T into S buffer j & 1 ------------------------------------------
@@ -432,10 +435,22 @@ __global__ void __launch_bounds__(kThreads, 2)
   }
   if constexpr (!kPrefix) pdl_launch_dependents();
   tc05::fence_before_sync();
-  __syncthreads();
+  const int any_fail = __syncthreads_or(!ok);
   if (warp == 5) {
     tc05::fence_after_sync();
     tc05::dealloc(tmem, kTmemCols);
+  }
+  if (any_fail && (warp == 4 || warp == 6) && lane == 0) {
+    // A wait gave up somewhere, so copies this producer issued may not have been consumed: give them
+    // a bounded chance to land before the CTA's shared memory goes. A stage is refilled only after
+    // its previous fill was consumed, so only the last fill of each stage can be outstanding, and
+    // the parity wait for that fill is exact.
+    const int ns = warp == 4 ? kKStages : kVStages;
+    const int full0 = warp == 4 ? kKFull0 : kVFull0;
+    const uint64_t drain_deadline = globaltimer_ns() + 100000000ull;
+    for (int j = max(0, issued - ns); j < issued; ++j)
+      mbar_wait_bounded(B(full0 + j % ns), (j / ns) & 1, drain_deadline);
+    if (warp == 4) mbar_wait_bounded(B(kQFull), 0, drain_deadline);
   }
 }
 
