@@ -116,6 +116,8 @@ void pa_decode_opts_init(pa_decode_opts* opts);
  *   k_scale, v_scale  dequantisation scales of an E4M3 cache (> 0, finite); ignored otherwise.
  *   Slots outside [-1, num_blocks * 16) are skipped and set PA_DEVERR_BAD_SLOT in the library's
  *   error word. Untouched slots keep their bytes. Two tokens with the same slot race.
+ *   Limits (else PA_ERR_UNSUPPORTED / PA_ERR_INVALID_ARG): D a multiple of 8, T < 2^31, the pool's
+ *   size in bytes below 2^63.
  * Source: vLLM notes page, "PagedAttention / Cache Engine" (the engine writes a position's data
  * into its page). T == 0 is a no-op.
  */
@@ -134,7 +136,9 @@ int pa_reshape_and_cache(const pa_tensor* key, const pa_tensor* value, const pa_
  *                 step by pa_reshape_and_cache). 0 gives an all-zero output row.
  *   scale         multiplies q.k before the softmax (typically 1/sqrt(D)).
  *   num_kv_heads  Hkv; must equal k_cache.shape[1] and divide Hq. Query head h reads KV head
- *                 h / (Hq / Hkv). Supported: D in {64, 128} (E4M3: 128), Hq / Hkv <= 16.
+ *                 h / (Hq / Hkv). Supported: D in {64, 128} (E4M3: 128), Hq / Hkv <= 16,
+ *                 B and Hkv <= 65535, num_blocks * Hkv * 16 < 2^31 pool rows (else
+ *                 PA_ERR_UNSUPPORTED). Block-table columns past 2^31 / 16 are never read.
  * out[s, h, :] = sum_t softmax_t(scale * q[s, h] . K[s, t]) V[s, t], K[s, t] being row t % 16 of
  * page (block_tables[s][t / 16], h / G); accumulation in float32, result rounded to nearest even.
  * The result depends only on logical positions, never on which physical blocks hold them.
