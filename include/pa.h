@@ -219,7 +219,7 @@ size_t pa_decode_cascade_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, 
  *   block_tables  [B, max_blocks] I32; query_start [B + 1] I32; context_lens [B] I32: tokens of
  *                 sequence s including the chunk (n_s <= context_lens[s] <= 16 * max_blocks).
  *   max_query_len host-known bound on n_s (sizes the grid without a device read).
- *   kernel        -1 = choose (tcgen05 when D = 128 and Hq / Hkv divides 128), 0 = warp-level mma.sync
+ *   kernel        -1 = choose (tcgen05 when D = 128 and Hq / Hkv <= 16 divides 128), 0 = warp-level mma.sync
  *                 tiles, 1 = tcgen05 (5th-generation tensor cores, accumulators in tensor memory).
  * Row i of sequence s is position p = context_lens[s] - n_s + i and sees positions 0 .. p:
  * out = softmax(scale * q K[0..p]^T) V[0..p], float32 accumulation, rounded to nearest even.

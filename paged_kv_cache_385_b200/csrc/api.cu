@@ -738,7 +738,7 @@ int pa_prefill(pa_tensor* out, const pa_tensor* q, const pa_tensor* k_cache, con
   const int G = static_cast<int>(Hq / num_kv_heads);
   if (kernel < -1 || kernel > 1) return fail(PA_ERR_INVALID_ARG, "kernel must be -1, 0 or 1");
   const bool tc_ok = pa::prefill_tc_supported(static_cast<int>(D), G);
-  if (kernel == 1 && !tc_ok) return fail(PA_ERR_UNSUPPORTED, "the tcgen05 prefill needs head_dim 128 and a group dividing 128");
+  if (kernel == 1 && !tc_ok) return fail(PA_ERR_UNSUPPORTED, "the tcgen05 prefill needs head_dim 128 and a group of at most 16 dividing 128");
   pa::MqParams p{};
   p.q = q->data;
   p.q_stride_s = q->stride[0];
