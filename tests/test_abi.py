@@ -419,3 +419,20 @@ def test_struct_layouts_match_the_header(tmp_path):
         assert int(got[f"{st_} size"]) == ctypes.sizeof(cls)
         for n in fields[st_]:
             assert int(got[f"{st_} {n}"]) == getattr(cls, n).offset, (st_, n)
+
+
+def test_measurement_probes_build(tmp_path):
+    """The stand-alone probes behind figures quoted beside the roofline still compile for sm_100a
+    (they share the library's device headers), and the Python one parses."""
+    import py_compile
+    import shutil
+    nvcc = shutil.which("nvcc") or "/usr/local/cuda/bin/nvcc"
+    if not os.path.exists(nvcc):
+        pytest.skip("no nvcc")
+    measure = os.path.join(ROOT, "paged_kv_cache_385_b200", "measure")
+    for src in sorted(f for f in os.listdir(measure) if f.endswith(".cu")):
+        subprocess.run([nvcc, "-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-std=c++17", "-I",
+                        os.path.join(ROOT, "include"), "-c", os.path.join(measure, src), "-o",
+                        str(tmp_path / (src + ".o"))], check=True, capture_output=True)
+    for src in sorted(f for f in os.listdir(measure) if f.endswith(".py")):
+        py_compile.compile(os.path.join(measure, src), cfile=str(tmp_path / (src + "c")), doraise=True)
