@@ -212,7 +212,10 @@ __global__ void __launch_bounds__(kThreads, 2)
       ok = mbar_wait_bounded(B(kQFull), 0, deadline);
       for (int j = 0; j < nkb && ok; ++j) {
         // Buffer j & 1 holds P(j-2) until P(j-2).V has completed. O_done's phases are waited in
-        // order (j - 2 = 0, 1, ...), so this parity wait cannot be taken for an older phase.
+        // order (j - 2 = 0, 1, ...), so this parity wait is never taken for an older phase. It would
+        // see O_done two phases ahead only if this thread stalled, between issuing QK(j-1) and its
+        // first poll here, for longer than QK(j-1), softmax(j-1) and P(j-1).V together; the wait
+        // would then give up at its bound (error bit). Per-parity O_done barriers would close that.
         const int ks_ = j % kKStages;
         if ((j >= 2 && !mbar_wait_bounded(B(kODone), (j - 2) & 1, deadline)) ||
             !mbar_wait_bounded(B(kKFull0 + ks_), (j / kKStages) & 1, deadline)) {
