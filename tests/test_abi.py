@@ -15,6 +15,7 @@ from hypothesis import strategies as st
 import paged_kv_cache_385_b200 as pa
 import workloads as W
 from oracle import paging
+from tests.host_buffers import aligned_zeros
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
@@ -148,20 +149,14 @@ def test_slot_helper_rejects_out_of_range():
     assert pa.pa_slots_for_positions(bt, [0], [5]).tolist() == [53]
 
 
-def _aligned_zeros(shape, dtype, align=256):
-    """A zeroed host tensor whose data starts on an `align`-byte boundary (the library checks it)."""
-    n = int(np.prod(shape)) * torch.tensor([], dtype=dtype).element_size()
-    raw = torch.zeros(n + align, dtype=torch.uint8)
-    off = (-raw.data_ptr()) % align
-    return raw[off:off + n].view(dtype).view(*shape)
 
 
 def test_cascade_option_validation_happens_on_the_host():
     """A bad opts.prefix_kernel or an unaligned prefix length is refused before any device work (the
     tensors here are host memory, which no kernel could read)."""
     B, Hq, Hkv, D, NB = 2, 8, 2, 128, 16
-    q = _aligned_zeros((B, Hq, D), torch.bfloat16)
-    kc = _aligned_zeros((NB, Hkv, 16, D), torch.bfloat16)
+    q = aligned_zeros((B, Hq, D), torch.bfloat16)
+    kc = aligned_zeros((NB, Hkv, 16, D), torch.bfloat16)
     bt = torch.zeros(B, 4, dtype=torch.int32)
     lens = torch.full((B,), 40, dtype=torch.int32)
     ts = [pa.as_pa_tensor(t, n, device=False) for t, n in ((q, "out"), (q, "q"), (kc, "k"), (kc, "v"), (bt, "bt"),
@@ -187,8 +182,8 @@ def test_prefill_kernel_choice_is_checked_on_the_host():
     """The tcgen05 prefill takes head_dim 128 and a group dividing 128: asking for it with D = 64 is
     refused before any device work; an unknown kernel number too."""
     T, Hq, Hkv, D, NB, B = 8, 4, 4, 64, 4, 1
-    q = _aligned_zeros((T, Hq, D), torch.float16)
-    kc = _aligned_zeros((NB, Hkv, 16, D), torch.float16)
+    q = aligned_zeros((T, Hq, D), torch.float16)
+    kc = aligned_zeros((NB, Hkv, 16, D), torch.float16)
     bt = torch.zeros(B, 1, dtype=torch.int32)
     qs = torch.tensor([0, T], dtype=torch.int32)
     lens = torch.tensor([T], dtype=torch.int32)
@@ -210,9 +205,9 @@ def test_decode_argument_errors_are_reported_before_device_work():
     """Every argument error of pa_decode is found on the host, the workspace check included: the
     tensors here are host memory, so a call that reached the device would not return these codes."""
     B, Hq, Hkv, D, NB = 2, 8, 2, 128, 16
-    q = _aligned_zeros((B, Hq, D), torch.bfloat16)
-    kc = _aligned_zeros((NB, Hkv, 16, D), torch.bfloat16)
-    kc16 = _aligned_zeros((NB, Hkv, 16, D), torch.float16)
+    q = aligned_zeros((B, Hq, D), torch.bfloat16)
+    kc = aligned_zeros((NB, Hkv, 16, D), torch.bfloat16)
+    kc16 = aligned_zeros((NB, Hkv, 16, D), torch.float16)
     bt = torch.zeros(B, 64, dtype=torch.int32)
     lens = torch.full((B,), 1000, dtype=torch.int32)
     lib = pa.lib()
@@ -234,9 +229,9 @@ def test_decode_argument_errors_are_reported_before_device_work():
     # A split into 1024 / 256 = 4 partitions needs a workspace; none given.
     assert call(partition_tokens=256) == pa.PA_ERR_WORKSPACE
     assert "workspace" in pa.pa_last_error()
-    small = _aligned_zeros((64,), torch.uint8)
+    small = aligned_zeros((64,), torch.uint8)
     assert call(partition_tokens=256, workspace=small.data_ptr(), workspace_bytes=64) == pa.PA_ERR_WORKSPACE
-    kc3 = _aligned_zeros((NB, 3, 16, D), torch.bfloat16)
+    kc3 = aligned_zeros((NB, 3, 16, D), torch.bfloat16)
     assert call(kcache=kc3, hkv=3) == pa.PA_ERR_INVALID_ARG  # 8 query heads over 3 KV heads
     assert "multiple" in pa.pa_last_error()
     # Misaligned pointers: q / out rows, the pool, the workspace.
@@ -249,7 +244,7 @@ def test_decode_argument_errors_are_reported_before_device_work():
         assert lib.pa_decode(*[ctypes.byref(t) for t in ts], 0.088, Hkv, ctypes.byref(opts), None) == \
             pa.PA_ERR_INVALID_ARG
         assert "aligned" in pa.pa_last_error()
-    big = _aligned_zeros((1 << 20,), torch.uint8)
+    big = aligned_zeros((1 << 20,), torch.uint8)
     assert call(partition_tokens=256, workspace=big.data_ptr() + 8, workspace_bytes=(1 << 20) - 8) == \
         pa.PA_ERR_INVALID_ARG
     assert "aligned" in pa.pa_last_error()
@@ -277,9 +272,9 @@ def test_no_alloc_decode_checks_arguments_before_the_scratch_lookup():
     """pa_decode_no_alloc finds argument errors, the scratch capacity included, before its first CUDA
     call (the lookup of the built-in array): with host tensors it returns them, not PA_ERR_CUDA."""
     B, Hkv, G, D = 64, 8, 8, 128
-    q = _aligned_zeros((B, Hkv * G, D), torch.bfloat16)
-    kc = _aligned_zeros((16, Hkv, 16, D), torch.bfloat16)
-    kc16 = _aligned_zeros((16, Hkv, 16, D), torch.float16)
+    q = aligned_zeros((B, Hkv * G, D), torch.bfloat16)
+    kc = aligned_zeros((16, Hkv, 16, D), torch.bfloat16)
+    kc16 = aligned_zeros((16, Hkv, 16, D), torch.float16)
     bt = torch.zeros(B, 8192, dtype=torch.int32)
     lens = torch.ones(B, dtype=torch.int32)
     lib = pa.lib()
@@ -298,7 +293,7 @@ def test_no_alloc_decode_checks_arguments_before_the_scratch_lookup():
     # 64 sequences x 64 heads x 512 partitions of 256 tokens: far more than the built-in array.
     assert call(max_context_len=8192 * 16, partition_tokens=256) == pa.PA_ERR_WORKSPACE
     assert "scratch" in pa.pa_last_error()
-    small = _aligned_zeros((256,), torch.uint8)
+    small = aligned_zeros((256,), torch.uint8)
     assert call(workspace=small.data_ptr(), workspace_bytes=256) == pa.PA_ERR_INVALID_ARG
 
 

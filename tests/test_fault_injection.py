@@ -12,23 +12,19 @@ import pytest
 import torch
 
 import paged_kv_cache_385_b200 as pa
+from tests.host_buffers import aligned_zeros
 
 pytestmark = pytest.mark.skipif(torch.cuda.is_available(),
                                 reason="host-pointer descriptors must never reach a GPU launch")
 
 
-def _aligned(shape, dtype, align=256):
-    n = int(np.prod(shape)) * torch.tensor([], dtype=dtype).element_size()
-    raw = torch.zeros(n + align, dtype=torch.uint8)
-    off = (-raw.data_ptr()) % align
-    return raw[off:off + n].view(dtype).view(*shape)
 
 
 @pytest.fixture
 def decode_args():
     B, Hq, Hkv, D, NB = 2, 8, 2, 128, 16
-    q = _aligned((B, Hq, D), torch.bfloat16)
-    kc = _aligned((NB, Hkv, 16, D), torch.bfloat16)
+    q = aligned_zeros((B, Hq, D), torch.bfloat16)
+    kc = aligned_zeros((NB, Hkv, 16, D), torch.bfloat16)
     bt = torch.zeros(B, 4, dtype=torch.int32)
     lens = torch.full((B,), 40, dtype=torch.int32)
     ts = [pa.as_pa_tensor(t, n, device=False) for t, n in ((q, "out"), (q, "q"), (kc, "k"), (kc, "v"), (bt, "bt"),
@@ -56,11 +52,11 @@ def test_injected_failures_are_counted_and_host_only(decode_args):
 
 def test_every_enqueuing_entry_point_takes_the_hook():
     T, Hkv, D, NB = 3, 2, 64, 8
-    key = _aligned((T, Hkv, D), torch.float16)
-    kc = _aligned((NB, Hkv, 16, D), torch.float16)
+    key = aligned_zeros((T, Hkv, D), torch.float16)
+    kc = aligned_zeros((NB, Hkv, 16, D), torch.float16)
     slots = torch.zeros(T, dtype=torch.int64)
     mapping = torch.tensor([[0, 1]], dtype=torch.int64)
-    q = _aligned((T, Hkv, D), torch.float16)
+    q = aligned_zeros((T, Hkv, D), torch.float16)
     bt = torch.zeros(1, 1, dtype=torch.int32)
     qs = torch.tensor([0, T], dtype=torch.int32)
     lens = torch.tensor([T], dtype=torch.int32)
@@ -105,15 +101,15 @@ def test_queried_workspace_size_is_exactly_what_the_call_checks(cascade):
         prefix = 16 * int(rng.integers(1, mb + 1)) if cascade else 0
         if cascade and D != 128:
             D = 128
-        q = _aligned((B, Hkv * G, D), torch.bfloat16)
-        kc = _aligned((4, Hkv, 16, D), torch.bfloat16)
+        q = aligned_zeros((B, Hkv * G, D), torch.bfloat16)
+        kc = aligned_zeros((4, Hkv, 16, D), torch.bfloat16)
         bt = torch.zeros(B, mb, dtype=torch.int32)
         lens = torch.ones(B, dtype=torch.int32)
         if cascade:
             need = pa.pa_decode_cascade_workspace_bytes(B, Hkv * G, Hkv, D, max_ctx, prefix, pt)
         else:
             need = pa.pa_decode_workspace_bytes(B, Hkv * G, Hkv, D, max_ctx, pt)
-        ws = _aligned((max(need, 1),), torch.uint8)
+        ws = aligned_zeros((max(need, 1),), torch.uint8)
         ts = [pa.as_pa_tensor(t, n, device=False) for t, n in ((q, "out"), (q, "q"), (kc, "k"), (kc, "v"),
                                                                 (bt, "bt"), (lens, "lens"))]
 
@@ -151,8 +147,8 @@ def test_no_alloc_accepts_exactly_the_batches_its_array_holds():
         Hkv, G = int(rng.choice([1, 8])), int(rng.choice([1, 8]))
         B, D, mb = int(rng.integers(1, 64)), 128, int(rng.integers(1, 8192))
         max_ctx, pt = int(rng.integers(1, mb * 16 + 1)), int(rng.choice([0, 256, 512]))
-        q = _aligned((B, Hkv * G, D), torch.bfloat16)
-        kc = _aligned((4, Hkv, 16, D), torch.bfloat16)
+        q = aligned_zeros((B, Hkv * G, D), torch.bfloat16)
+        kc = aligned_zeros((4, Hkv, 16, D), torch.bfloat16)
         bt, lens = torch.zeros(B, mb, dtype=torch.int32), torch.ones(B, dtype=torch.int32)
         ts = [pa.as_pa_tensor(t, n, device=False) for t, n in ((q, "out"), (q, "q"), (kc, "k"), (kc, "v"),
                                                                 (bt, "bt"), (lens, "lens"))]
