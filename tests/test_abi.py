@@ -149,8 +149,6 @@ def test_slot_helper_rejects_out_of_range():
     assert pa.pa_slots_for_positions(bt, [0], [5]).tolist() == [53]
 
 
-
-
 def test_cascade_option_validation_happens_on_the_host():
     """A bad opts.prefix_kernel or an unaligned prefix length is refused before any device work (the
     tensors here are host memory, which no kernel could read)."""

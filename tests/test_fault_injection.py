@@ -18,8 +18,6 @@ pytestmark = pytest.mark.skipif(torch.cuda.is_available(),
                                 reason="host-pointer descriptors must never reach a GPU launch")
 
 
-
-
 @pytest.fixture
 def decode_args():
     B, Hq, Hkv, D, NB = 2, 8, 2, 128, 16
