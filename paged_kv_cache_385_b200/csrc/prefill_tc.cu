@@ -57,9 +57,9 @@ enum {
   kVEmpty0 = 9,  // kVStages
   kSFull0 = 11,  // 2
   kPFull0 = 13,  // 2: block j arrives on kPFull0 + (j & 1)
-  kODone = 15,
-  kAllDone = 16,
-  kTmemSlot = 17,
+  kODone0 = 15,  // 2: P(j).V commits to kODone0 + (j & 1)
+  kAllDone = 17,
+  kTmemSlot = 18,
 };
 static_assert(8 * (kTmemSlot + 1) <= 256, "barrier area");
 // O is rescaled only when a row's running max grows by more than this (log2 units); until then P and
@@ -143,7 +143,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     mbar_init(B(kSFull0 + 1), 1);
     mbar_init(B(kPFull0), 4);
     mbar_init(B(kPFull0 + 1), 4);
-    mbar_init(B(kODone), 1);
+    mbar_init(B(kODone0), 1);
+    mbar_init(B(kODone0 + 1), 1);
     mbar_init(B(kAllDone), 1);
     fence_barrier_init();
   }
@@ -211,13 +212,12 @@ __global__ void __launch_bounds__(kThreads, 2)
       constexpr uint32_t idesc_qk = tc05::idesc_f16(kBf16, kRows, kKeys, false, false);
       ok = mbar_wait_bounded(B(kQFull), 0, deadline);
       for (int j = 0; j < nkb && ok; ++j) {
-        // Buffer j & 1 holds P(j-2) until P(j-2).V has completed. O_done's phases are waited in
-        // order (j - 2 = 0, 1, ...), so this parity wait is never taken for an older phase. It would
-        // see O_done two phases ahead only if this thread stalled, between issuing QK(j-1) and its
-        // first poll here, for longer than QK(j-1), softmax(j-1) and P(j-1).V together; the wait
-        // would then give up at its bound (error bit). Per-parity O_done barriers would close that.
+        // Buffer j & 1 holds P(j-2) until P(j-2).V has completed. O_done is two barriers by block
+        // parity, so the one waited here next completes for P(j).V, which needs S(j) from the QK this
+        // thread has yet to issue: the barrier cannot be two phases ahead. Nor one behind: QK(j-2)
+        // was issued only after P(j-4).V completed on it.
         const int ks_ = j % kKStages;
-        if ((j >= 2 && !mbar_wait_bounded(B(kODone), (j - 2) & 1, deadline)) ||
+        if ((j >= 2 && !mbar_wait_bounded(B(kODone0 + (j & 1)), ((j - 2) >> 1) & 1, deadline)) ||
             !mbar_wait_bounded(B(kKFull0 + ks_), (j / kKStages) & 1, deadline)) {
           ok = false;
           break;
@@ -259,7 +259,7 @@ __global__ void __launch_bounds__(kThreads, 2)
           tc05::mma_f16_ts(tO, tS0 + (j & 1) * kKeys + kt * 8, tc05::smem_desc_sw128(vbase + kt * 2048, kHalfKV, 1024),
                            idesc_pv, (j > 0 || kt > 0));
         }
-        tc05::commit(B(kODone));
+        tc05::commit(B(kODone0 + (j & 1)));
         tc05::commit(B(kVEmpty0 + j % kVStages));
       }
       // Every QK has completed before its softmax finished, so this covers all of the CTA's MMAs.
@@ -332,9 +332,11 @@ __global__ void __launch_bounds__(kThreads, 2)
         rs[(2 * k + 1) & 3] += p1;
       }
       l = l * alpha + ((rs[0] + rs[1]) + (rs[2] + rs[3]));
-      // O's rescale waits for the previous P . V (only when the reference moved).
+      // O's rescale waits for the previous P . V (only when the reference moved). Its barrier next
+      // completes for P(j+1).V, which needs this warp's P(j+1): never two phases ahead. It is not
+      // one behind either: S(j-1) came from QK(j-1), issued after P(j-3).V completed on it.
       if (raise && j > 0) {
-        const bool done = mbar_wait_bounded(B(kODone), (j - 1) & 1, deadline);
+        const bool done = mbar_wait_bounded(B(kODone0 + ((j - 1) & 1)), ((j - 1) >> 1) & 1, deadline);
         if (!__all_sync(kFull, done)) {
           ok = false;
           break;

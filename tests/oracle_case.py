@@ -98,3 +98,33 @@ def expected_out_paged(case: OracleCase) -> np.ndarray:
     w = case.w
     return attention.decode_paged(case.q, case.k_pool, case.v_pool, case.block_tables, case.lens, w.scale,
                                   w.num_kv_heads, w.kv_dtype, case.k_scale, case.v_scale, w.block_size)
+
+
+def _all_bf16_values() -> np.ndarray:
+    """Every bf16 bit pattern 0 .. 65535, as the float32 value it holds (index = bit pattern)."""
+    bits = np.arange(65536, dtype=np.uint32) << 16
+    return bits.view(np.float32)
+
+
+_CODE_TABLES = {}
+
+
+def e4m3_codes_of_bf16(src: torch.Tensor, scale: float) -> np.ndarray:
+    """``oracle.e4m3.quantize(src, scale)`` for a bf16 source, looked up by the source's bits.
+
+    quantize acts on each element alone, and a bf16 element holds one of 65536 bit patterns, so
+    evaluating quantize once on every pattern and indexing that table by the source's bits gives
+    exactly quantize's codes (``tests/test_oracle_e4m3.py`` checks the two agree). Full-size workloads
+    hold ~10^9 elements, which the element-wise codec would take many minutes over.
+    """
+    assert src.dtype == torch.bfloat16
+    key = float(scale)
+    if key not in _CODE_TABLES:
+        _CODE_TABLES[key] = e4m3.quantize(_all_bf16_values(), scale)
+    return _CODE_TABLES[key][bits16(src)]
+
+
+def e4m3_values(codes: np.ndarray, scale: float) -> np.ndarray:
+    """``oracle.e4m3.dequantize(codes, scale)`` by lookup in its value at each of the 256 codes."""
+    table = e4m3.dequantize(np.arange(256, dtype=np.uint8), scale)
+    return table[codes]

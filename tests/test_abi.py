@@ -414,18 +414,9 @@ def test_struct_layouts_match_the_header(tmp_path):
             assert int(got[f"{st_} {n}"]) == getattr(cls, n).offset, (st_, n)
 
 
-def test_measurement_probes_build(tmp_path):
-    """The stand-alone probes behind figures quoted beside the roofline still compile for sm_100a
-    (they share the library's device headers), and the Python one parses."""
-    import py_compile
-    import shutil
-    nvcc = shutil.which("nvcc") or "/usr/local/cuda/bin/nvcc"
-    if not os.path.exists(nvcc):
-        pytest.skip("no nvcc")
-    measure = os.path.join(ROOT, "paged_kv_cache_385_b200", "measure")
-    for src in sorted(f for f in os.listdir(measure) if f.endswith(".cu")):
-        subprocess.run([nvcc, "-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-std=c++17", "-I",
-                        os.path.join(ROOT, "include"), "-c", os.path.join(measure, src), "-o",
-                        str(tmp_path / (src + ".o"))], check=True, capture_output=True)
-    for src in sorted(f for f in os.listdir(measure) if f.endswith(".py")):
-        py_compile.compile(os.path.join(measure, src), cfile=str(tmp_path / (src + "c")), doraise=True)
+def test_no_alloc_scratch_size_matches_the_header():
+    """The binding's NO_ALLOC_SCRATCH_BYTES is the header's PA_NO_ALLOC_SCRATCH_BYTES."""
+    text = open(os.path.join(ROOT, "include", "pa.h")).read()
+    m = re.search(r"#define PA_NO_ALLOC_SCRATCH_BYTES \(\(size_t\)(\d+) << (\d+)\)", text)
+    assert m, "PA_NO_ALLOC_SCRATCH_BYTES is not defined as ((size_t)a << b)"
+    assert pa.NO_ALLOC_SCRATCH_BYTES == int(m.group(1)) << int(m.group(2))

@@ -157,20 +157,49 @@ def test_cascade_reports_a_table_without_the_shared_prefix(prefix_kernel):
 
 
 @pytest.mark.parametrize("prefix_kernel", PREFIX_KERNELS)
-def test_full_size_prefix_workload_sampled(prefix_kernel):
-    from oracle import attention
-    w = W.FULL["prefix_gqa"]
-    dev = DeviceCase(w, sentinel=False)
-    out = dev.cascade(fused=True, prefix_kernel=prefix_kernel).cpu()
+@pytest.mark.parametrize("fused", [True, False])
+def test_permuted_physical_blocks_give_bit_identical_cascade(fused, prefix_kernel):
+    """Two free-list orders place the shared prefix and every suffix in different physical blocks;
+    the cascade output (prefix kernel, suffix decode and merge) must not change by a bit."""
+    w = W.ALL["prefix_gqa_small"]
+    outs, tables = [], []
+    for seed in (21, 22):
+        order = torch.randperm(w.num_blocks, generator=torch.Generator().manual_seed(seed)).to(torch.int32)
+        dev = DeviceCase(w, order=order)
+        if not fused:
+            dev.write_new_token()
+        for pt in (0, 16):
+            outs.append((pt, dev.cascade(fused=fused, partition_tokens=pt, prefix_kernel=prefix_kernel).clone()))
+        tables.append(dev.bt_host)
+    torch.cuda.synchronize()
     assert pa.pa_read_device_error(clear=True) == 0
-    lens = dev.lens_host
-    rng = np.random.default_rng(11)
-    worst = 0.0
-    for s in sorted(set(rng.integers(0, w.num_seqs, 6).tolist())):
-        K = W.kv_source(w, s, "k", lens).double().numpy()
-        V = W.kv_source(w, s, "v", lens).double().numpy()
-        q = W.query(w)[s].double().numpy()
-        for h in (0, 5, 31):
-            want = attention.decode_logical_one(q[h], K, V, h, w.num_q_heads, w.num_kv_heads, w.scale)
-            worst = max(worst, float(np.max(np.abs(out[s, h].double().numpy() - want))))
-    assert worst <= TOL[w.kv_dtype], worst
+    assert not torch.equal(tables[0], tables[1])
+    for pt in (0, 16):
+        a, b = [o for p, o in outs if p == pt]
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16)), pt
+
+
+@pytest.mark.parametrize("prefix_kernel", PREFIX_KERNELS)
+def test_permuted_prefix_of_several_chunks_is_bit_identical(prefix_kernel):
+    """The 640-token, two-row-tile case with its blocks renumbered by a random permutation."""
+    rng = np.random.default_rng(8)
+    lens = [int(x) for x in 640 + rng.integers(1, 120, 40)]
+    lens[3], lens[30] = 300, 17
+    q, kc, vc, bt = _shared_prefix_case(lens, 8, 2, 640, torch.bfloat16, seed=641)
+    perm = torch.randperm(kc.shape[0], generator=torch.Generator().manual_seed(9))
+    # Block b moves to perm[b]: the same logical data in other physical blocks.
+    kc2, vc2 = torch.empty_like(kc), torch.empty_like(vc)
+    kc2[perm], vc2[perm] = kc, vc
+    bt2 = torch.where(bt >= 0, perm[bt.clamp(min=0).long()].to(torch.int32), bt)
+    n = pa.pa_decode_cascade_workspace_bytes(len(lens), 8, 2, 128, max(lens), 640, 0)
+    ws = torch.empty(n, dtype=torch.uint8, device="cuda")
+    outs = []
+    for k_, v_, t_ in ((kc, vc, bt), (kc2, vc2, bt2)):
+        out = torch.empty(len(lens), 8, 128, dtype=torch.bfloat16, device="cuda")
+        pa.pa_decode_cascade(out, q.cuda(), None, None, None, k_.cuda(), v_.cuda(), t_.cuda(),
+                             torch.tensor(lens, dtype=torch.int32).cuda(), 640, 0.0884, 2, workspace=ws,
+                             max_context_len=max(lens), prefix_kernel=prefix_kernel)
+        outs.append(out)
+    torch.cuda.synchronize()
+    assert pa.pa_read_device_error(clear=True) == 0
+    assert torch.equal(outs[0].view(torch.int16), outs[1].view(torch.int16))

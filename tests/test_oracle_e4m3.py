@@ -96,3 +96,18 @@ def test_quantize_is_float32_multiply_then_encode():
         prod = torch.from_numpy(x) * inv
         ref = prod.clamp(-448, 448).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
         assert np.array_equal(e4m3.quantize(x, scale), ref)
+
+
+def test_tabulated_quantize_equals_the_codec():
+    """The full-size GPU tests look the oracle's codes up in quantize's value on every bf16 pattern;
+    that lookup must equal quantize applied element by element (random draws, the extremes, NaN/inf)."""
+    from tests import oracle_case
+    g = torch.Generator().manual_seed(3)
+    src = torch.cat([torch.randn(200000, generator=g) * 3, torch.tensor([0.0, -0.0, 1e30, -1e30, 448.0, 500.0,
+                                                                          float("inf"), float("nan")])])
+    src = src.to(torch.bfloat16)
+    for scale in (5.5 / 448, 1.0, 0.013):
+        direct = e4m3.quantize(src.float().numpy(), scale)
+        assert np.array_equal(oracle_case.e4m3_codes_of_bf16(src, scale), direct)
+        assert np.array_equal(oracle_case.e4m3_values(direct, scale), e4m3.dequantize(direct, scale),
+                              equal_nan=True)
