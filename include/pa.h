@@ -346,6 +346,22 @@ int pa_blocks_alloc_n(pa_allocator* a, int32_t n, int32_t* out);
 int pa_blocks_incref_n(pa_allocator* a, int32_t n, const int32_t* blocks);
 int pa_blocks_free_n(pa_allocator* a, int32_t n, const int32_t* blocks);
 
+/* Block tables of a batch, built with the allocator: out is host I32 [num_seqs, max_blocks] (row
+ * stride max_blocks), entries past ceil(context_lens[s] / 16) set to -1. Sequences are served in
+ * order and each logical block in order: logical block j of sequence s gets a block popped from the
+ * free list, except that the first shared_prefix_tokens / 16 logical blocks are shared by every
+ * sequence reaching them: each is allocated by the first sequence that reaches it, and every later
+ * one takes a reference to it (a sequence shorter than the prefix shares only the blocks it covers).
+ *   context_lens  host I32 [num_seqs], >= 0; shared_prefix_tokens a multiple of 16 (0 = none).
+ * All-or-nothing: PA_ERR_EXHAUSTED (nothing allocated, out untouched) if the free list holds fewer
+ * blocks than the tables need; PA_ERR_INVALID_ARG (nothing changed) for a negative length, a
+ * sequence needing more than max_blocks blocks, or a bad prefix length.
+ * Source: vLLM notes page, "PagedAttention / Block Manager" (blocks handed out from a free list as
+ * a request needs them) and "vLLM 前世今生" section 3.2 (non-contiguous physical blocks mapped by a
+ * block table; sequences sharing a prompt prefix point at the same physical blocks). */
+int pa_build_block_tables(pa_allocator* a, const int32_t* context_lens, int32_t num_seqs, int32_t max_blocks,
+                          int32_t shared_prefix_tokens, int32_t* out);
+
 /* Host helper: slot of each (sequence, position) pair, slot = bt[seq][pos / 16] * 16 + pos % 16.
  *   block_tables  host I32, num_seqs rows of row_stride elements, max_blocks valid entries each.
  *   token_seq, token_pos, slots_out  host arrays of num_tokens entries.

@@ -104,6 +104,7 @@ def _load() -> ctypes.CDLL:
         "pa_blocks_alloc_n": (ctypes.c_int, [VP, I32, i32p]),
         "pa_blocks_incref_n": (ctypes.c_int, [VP, I32, i32p]),
         "pa_blocks_free_n": (ctypes.c_int, [VP, I32, i32p]),
+        "pa_build_block_tables": (ctypes.c_int, [VP, i32p, I32, I32, I32, i32p]),
         "pa_slots_for_positions": (ctypes.c_int, [i32p, I64, I32, I32, i32p, i32p, I64,
                                                   ctypes.POINTER(ctypes.c_int64)]),
     }
@@ -432,27 +433,11 @@ class BlockAllocator:
 
 def build_block_tables(alloc: BlockAllocator, context_lens: Sequence[int], max_blocks: int,
                        shared_prefix_tokens: int = 0) -> torch.Tensor:
-    """Host int32 block tables [num_seqs, max_blocks] (-1 padded) from the allocator.
-
-    Sequences are served in order, one allocation per logical block. With a shared prefix (a whole
-    number of blocks) each prefix block is allocated by the first sequence that reaches it, and
-    every later sequence reaching it takes a reference to it.
-    """
-    if shared_prefix_tokens % BLOCK_SIZE:
-        raise ValueError("shared_prefix_tokens must be a multiple of 16")
-    npre = shared_prefix_tokens // BLOCK_SIZE
-    lens = [int(c) for c in context_lens]
-    bt = torch.full((len(lens), max_blocks), -1, dtype=torch.int32)
-    prefix = torch.empty(0, dtype=torch.int32)  # prefix blocks allocated so far
-    for s, n in enumerate(lens):
-        nb = -(-n // BLOCK_SIZE)
-        if nb > max_blocks:
-            raise ValueError(f"sequence {s} needs {nb} blocks > max_blocks {max_blocks}")
-        reuse = min(npre, nb, prefix.numel())
-        if reuse:
-            alloc.incref_n(prefix[:reuse])
-        row = torch.cat([prefix[:reuse], alloc.alloc_n(nb - reuse)])
-        if min(npre, nb) > prefix.numel():
-            prefix = row[:min(npre, nb)].clone()
-        bt[s, :nb] = row
+    """Host int32 block tables [num_seqs, max_blocks] (-1 padded) from the allocator
+    (``pa_build_block_tables`` in include/pa.h: sequences in order, one allocation per logical block,
+    shared-prefix blocks allocated by the first sequence reaching them and referenced by later ones)."""
+    lens = torch.as_tensor([int(c) for c in context_lens], dtype=torch.int32).contiguous()
+    bt = torch.empty((lens.numel(), int(max_blocks)), dtype=torch.int32)
+    _check(_lib.pa_build_block_tables(alloc._h, _i32_ptr(lens), lens.numel(), int(max_blocks),
+                                      int(shared_prefix_tokens), _i32_ptr(bt)), "pa_build_block_tables")
     return bt

@@ -178,6 +178,59 @@ int pa_blocks_free_n(pa_allocator* a, int32_t n, const int32_t* blocks) {
   return PA_OK;
 }
 
+int pa_build_block_tables(pa_allocator* a, const int32_t* context_lens, int32_t num_seqs, int32_t max_blocks,
+                          int32_t shared_prefix_tokens, int32_t* out) {
+  if (!a || num_seqs < 0 || max_blocks < 0 || (num_seqs > 0 && (!context_lens || !out)))
+    return set_last_error(PA_ERR_INVALID_ARG, "NULL allocator, lengths or output, or a negative count");
+  if (shared_prefix_tokens < 0 || shared_prefix_tokens % PA_BLOCK_SIZE)
+    return set_last_error(PA_ERR_INVALID_ARG, "shared_prefix_tokens must be a non-negative multiple of %d (got %d)",
+                          PA_BLOCK_SIZE, shared_prefix_tokens);
+  const int32_t npre = shared_prefix_tokens / PA_BLOCK_SIZE;
+  // Count the allocations first (all-or-nothing): each sequence's own blocks past the prefix, plus
+  // the prefix blocks, each allocated once by the first sequence that reaches it.
+  int64_t fresh = 0;
+  int32_t prefix_reach = 0;
+  for (int32_t s = 0; s < num_seqs; ++s) {
+    const int32_t n = context_lens[s];
+    if (n < 0) return set_last_error(PA_ERR_INVALID_ARG, "context_lens[%d] is %d", s, n);
+    const int32_t nb = n / PA_BLOCK_SIZE + (n % PA_BLOCK_SIZE != 0);
+    if (nb > max_blocks)
+      return set_last_error(PA_ERR_INVALID_ARG, "sequence %d needs %d blocks, the table has %d", s, nb, max_blocks);
+    const int32_t in_prefix = std::min(npre, nb);
+    fresh += nb - in_prefix;
+    prefix_reach = std::max(prefix_reach, in_prefix);
+  }
+  fresh += prefix_reach;
+  if (fresh > static_cast<int64_t>(a->stack.size()))
+    return set_last_error(PA_ERR_EXHAUSTED, "the tables need %lld fresh blocks, %zu are free",
+                          static_cast<long long>(fresh), a->stack.size());
+  // Sequences in order, logical blocks in order: a prefix block already held is shared (one more
+  // reference), anything else is popped from the free list. At most num_seqs references per
+  // prefix block, so no count can overflow.
+  std::vector<int32_t> prefix;
+  try {
+    prefix.reserve(static_cast<size_t>(prefix_reach));
+  } catch (...) {
+    return set_last_error(PA_ERR_INVALID_ARG, "out of host memory");
+  }
+  for (int32_t s = 0; s < num_seqs; ++s) {
+    const int32_t n = context_lens[s];
+    const int32_t nb = n / PA_BLOCK_SIZE + (n % PA_BLOCK_SIZE != 0);
+    int32_t* row = out + static_cast<int64_t>(s) * max_blocks;
+    for (int32_t j = 0; j < nb; ++j) {
+      if (j < npre && j < static_cast<int32_t>(prefix.size())) {
+        row[j] = prefix[j];
+        ++a->ref[prefix[j]];
+      } else {
+        row[j] = pa_block_alloc(a);
+        if (j < npre) prefix.push_back(row[j]);
+      }
+    }
+    for (int32_t j = nb; j < max_blocks; ++j) row[j] = -1;
+  }
+  return PA_OK;
+}
+
 int pa_slots_for_positions(const int32_t* bt, int64_t row_stride, int32_t num_seqs, int32_t max_blocks,
                            const int32_t* token_seq, const int32_t* token_pos, int64_t num_tokens, int64_t* out) {
   if (num_tokens < 0 || (num_tokens > 0 && (!bt || !token_seq || !token_pos || !out)) || num_seqs < 0 ||

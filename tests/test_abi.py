@@ -266,6 +266,47 @@ def test_shared_prefix_blocks_come_from_the_first_sequence_reaching_them():
     assert alloc.num_free == nb - len(distinct)
 
 
+@settings(max_examples=120, deadline=None)
+@given(lens=st.lists(st.integers(0, 90), min_size=0, max_size=9), npre=st.integers(0, 5),
+       spare=st.integers(-3, 4), seed=st.integers(0, 2**31 - 1))
+def test_build_block_tables_through_the_c_abi(lens, npre, spare, seed):
+    """pa_build_block_tables called through ctypes with host arrays: the oracle's tables when the pool
+    suffices; otherwise PA_ERR_EXHAUSTED with the allocator and the output untouched."""
+    need = [-(-n // 16) for n in lens]
+    fresh = sum(max(0, b - npre) for b in need) + max([min(npre, b) for b in need] or [0])
+    nb = max(1, fresh + spare)
+    mb = max(need or [0]) + 1
+    order = np.random.default_rng(seed).permutation(nb).astype(np.int32)
+    alloc = pa.BlockAllocator(nb, order.tolist())
+    lens_a = np.ascontiguousarray(lens, dtype=np.int32)
+    out = np.full((len(lens), mb), 12345, dtype=np.int32)
+    i32p = ctypes.POINTER(ctypes.c_int32)
+    r = pa.lib().pa_build_block_tables(alloc._h, lens_a.ctypes.data_as(i32p), len(lens), mb, 16 * npre,
+                                       out.ctypes.data_as(i32p))
+    if fresh <= nb:
+        assert r == pa.PA_OK
+        want = paging.build_block_tables(lens, order, nb, 16, 16 * npre, mb) if lens else out[:0]
+        assert np.array_equal(out, want)
+        assert alloc.num_free == nb - fresh
+    else:
+        assert r == pa.PA_ERR_EXHAUSTED and "free" in pa.pa_last_error()
+        assert alloc.num_free == nb and (out == 12345).all()
+
+
+def test_build_block_tables_rejects_bad_arguments():
+    alloc = pa.BlockAllocator(64)
+    with pytest.raises(pa.PagedAttentionError) as e:
+        pa.build_block_tables(alloc, [10, 40], 2)  # 40 tokens need 3 blocks
+    assert e.value.status == pa.PA_ERR_INVALID_ARG
+    with pytest.raises(pa.PagedAttentionError) as e:
+        pa.build_block_tables(alloc, [10, -1], 2)
+    assert e.value.status == pa.PA_ERR_INVALID_ARG
+    with pytest.raises(pa.PagedAttentionError) as e:
+        pa.build_block_tables(alloc, [10], 2, shared_prefix_tokens=8)
+    assert e.value.status == pa.PA_ERR_INVALID_ARG
+    assert alloc.num_free == 64  # nothing was allocated by the refused calls
+
+
 def test_no_alloc_decode_checks_arguments_before_the_scratch_lookup():
     """pa_decode_no_alloc finds argument errors, the scratch capacity included, before its first CUDA
     call (the lookup of the built-in array): with host tensors it returns them, not PA_ERR_CUDA."""
