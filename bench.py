@@ -48,7 +48,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="llama7b_mha", choices=sorted(W.FULL))
-    ap.add_argument("--kernel", type=int, default=-1, help="-1 library choice, 0 CUDA-core, 1 tensor-core")
+    ap.add_argument("--kernel", type=int, default=-1,
+                    help="-1 library choice, 0 CUDA-core, 1 tensor-core, 2 tensor-core with one CTA per partition")
     ap.add_argument("--partition-tokens", type=int, default=None)
     ap.add_argument("--step", choices=["fused", "separate", "cascade"], default="fused",
                     help="fused: pa_decode_step (new-token write inside the decode launch); "
@@ -521,7 +522,7 @@ def run_ours(args, rank, world, local_rank):
                    "num_kv_heads": w.num_kv_heads, "head_dim": w.head_dim, "block_size": w.block_size,
                    "context_lens": "fixed 2048" if w.name == "llama7b_mha" else str(w.ctx),
                    "pool_blocks": w.num_blocks, "kv_bytes_per_step": kv_bytes,
-                   "partition_tokens": st.partition_tokens_used, "kernel": "tensor-core" if args.kernel != 0 else "cuda-core",
+                   "partition_tokens": st.partition_tokens_used, "kernel": {0: "cuda-core", 2: "tensor-core, one CTA per partition"}.get(args.kernel, "tensor-core"),
                    **({"prefix_kernel": "warp-level mma" if args.prefix_kernel == 0 else "tcgen05"}
                       if st.cascade_step else {}),
                    "l2": f"inputs larger than L2: {kv_bytes / 1e9:.2f} GB of KV per step vs 126 MB L2, no flush",

@@ -95,7 +95,10 @@ typedef struct pa_decode_opts {
   void* workspace;          /* device scratch for split partitions, >= pa_decode_workspace_bytes, 256-B
                                aligned; may be NULL when no split happens                               */
   size_t workspace_bytes;
-  int32_t kernel;           /* -1 = choose; 0 = CUDA-core FMA kernel; 1 = tensor-core (mma) kernel     */
+  int32_t kernel;           /* -1 = choose (1); 0 = CUDA-core FMA kernel; 1 = tensor-core (mma) kernel,
+                               whose split form (partitions of <= 512 tokens, <= 512 sequences, not
+                               the cascade suffix) runs one persistent warp per partition; 2 = the
+                               tensor-core kernel with one CTA per partition always                    */
   int32_t* error_word;      /* device int32 that receives PA_DEVERR_* bits; NULL = library's own word  */
   int32_t prefix_kernel;    /* pa_decode_cascade's shared-prefix kernel: -1 = choose (tcgen05 when
                                head_dim is 128, the group divides 128 and q rows are 16-B aligned);

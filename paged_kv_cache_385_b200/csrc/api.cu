@@ -415,8 +415,10 @@ static int decode_impl(pa_tensor* out, const pa_tensor* q, const pa_tensor* k_ca
   cfg.q = q->dtype == PA_BF16 ? pa::QType::BF16 : pa::QType::F16;
   cfg.head_dim = static_cast<int>(D);
   cfg.ntiles = static_cast<int>((G + 7) / 8);
-  cfg.kernel = opts.kernel < 0 ? 1 : opts.kernel;
-  if (cfg.kernel != 0 && cfg.kernel != 1) return fail(PA_ERR_INVALID_ARG, "opts.kernel must be -1, 0 or 1");
+  if (opts.kernel < -1 || opts.kernel > 2) return fail(PA_ERR_INVALID_ARG, "opts.kernel must be -1, 0, 1 or 2");
+  // 2: the tensor-core kernel, always one CTA per partition (no persistent per-warp split form).
+  const bool cta_per_partition = opts.kernel == 2;
+  cfg.kernel = opts.kernel < 0 || opts.kernel == 2 ? 1 : opts.kernel;
   if (!pa::decode_supported(cfg))
     return fail(PA_ERR_UNSUPPORTED, "no kernel for head_dim %lld, cache %s, q %s, group %lld, kernel %d", (long long)D,
                 dtype_name(cd), dtype_name(q->dtype), (long long)G, cfg.kernel);
@@ -596,7 +598,10 @@ static int decode_impl(pa_tensor* out, const pa_tensor* q, const pa_tensor* k_ca
     }
     if (e != cudaSuccess) return fail(PA_ERR_CUDA, "prefix launch: %s", cudaGetErrorString(e));
   }
-  e = pa::launch_decode(cfg, km, vm, p, s);
+  if (ws_parts > 1 && !cta_per_partition && pa::decode_units_supported(cfg, p))
+    e = pa::launch_decode_units(cfg, km, vm, p, s);
+  else
+    e = pa::launch_decode(cfg, km, vm, p, s);
   if (e != cudaSuccess) return fail(PA_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
   if (ws_parts > 1 && !p.merge_prefix_inline) {
     e = pa::launch_reduce(cfg, p, s);

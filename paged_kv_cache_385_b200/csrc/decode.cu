@@ -34,9 +34,11 @@
 //    partials, which they fold into their own merge (or leave to reduce_kernel when the suffix
 //    itself is split). The CTA of KV head 0, partition 0 of each sequence checks that its table
 //    maps the prefix to sequence 0's blocks.
+#include <algorithm>
 #include <cfloat>
 #include <utility>
 
+#include "decode_math.cuh"
 #include "internal.h"
 #include "pa_device.cuh"
 
@@ -47,261 +49,6 @@ __device__ uint32_t g_error_word;
 namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;
-
-// OCC is the number of CTAs per SM a kernel is compiled for: the page pipeline gets 192 KB / OCC of
-// shared memory (96, 64 or 48 KB) and registers are capped to fit. 16-bit pages with one query per
-// KV head are pure bandwidth: deep pipelines, 2 CTAs/SM. Grouped queries add math per byte and
-// e4m3 pages even more (widening, 3x the pages per byte moved), so those trade stages for resident
-// warps: 3 and 4 CTAs/SM.
-template <KvType KV, QType QT, int D, int NT, int KIND, int OCC>
-struct Cfg {
-  static constexpr bool kFp8 = KV == KvType::E4M3;
-  static constexpr int kEsz = kFp8 ? 1 : 2;
-  static constexpr int kRowBytes = D * kEsz;         // one token row of a page
-  static constexpr int kSubPages = kRowBytes / 128;  // 128-byte swizzled sub-pages per page
-  static constexpr int kSubElems = 128 / kEsz;       // TMA box width in elements
-  static constexpr int kPageBytes = 16 * kRowBytes;
-  static constexpr int kWarps = kDecodeWarps;
-  static constexpr int kThreads = kWarps * 32;
-  static constexpr int kStageBytes = 2 * kPageBytes;  // K page + V page
-  static constexpr int kMinBlocks = OCC;
-  static constexpr int kPipeBudget = OCC == 2 ? 96 * 1024 : (OCC == 3 ? 64 * 1024 : 48 * 1024);
-  static constexpr int kStages = kPipeBudget / (kWarps * kStageBytes);
-  static constexpr int kPipeBytes = kWarps * kStages * kStageBytes;
-  static constexpr bool kMmaBf16 = KV == KvType::BF16;  // e4m3 pages are widened to f16
-  static constexpr bool kQBf16 = QT == QType::BF16;
-  static constexpr int kGPad = 8 * NT;
-  static constexpr int kMergeFloats = kWarps * kGPad * (D + 2);
-  static constexpr int kSmemBytes = 1024 + kPipeBytes + kWarps * kStages * 8;
-  static_assert(kSubPages >= 1 && kRowBytes % 128 == 0, "page rows must be whole 128-byte lines");
-  static_assert(kStages >= 2, "need at least two stages per warp");
-  static_assert(kMergeFloats * 4 <= kPipeBytes, "merge area must fit in the pipeline buffers");
-};
-
-// Byte offset of 16-byte chunk `chunk` of token row `tok` in a 128-byte-swizzled sub-page.
-__device__ __forceinline__ uint32_t swz(int tok, int chunk) {
-  return static_cast<uint32_t>(tok * 128 + ((chunk ^ (tok & 7)) << 4));
-}
-
-template <class C>
-__device__ __forceinline__ uint32_t q_pair(const void* qrow, int d) {
-  // Two consecutive query elements (d, d+1) as the mma operand type.
-  const uint32_t raw = *reinterpret_cast<const uint32_t*>(static_cast<const uint16_t*>(qrow) + d);
-  if constexpr (C::kFp8 && C::kQBf16) {
-    const float2 f = unpack2<true>(raw);
-    return pack2<false>(f.x, f.y);
-  } else {
-    return raw;
-  }
-}
-
-// ---------------------------------------------------------------------------------------------
-// Tensor-core per-page math.
-// ---------------------------------------------------------------------------------------------
-template <class C, int D, int NT>
-struct TcMath {
-  static constexpr int KS = D / 16;  // k-steps of QK^T == m-tiles of PV
-  uint32_t qf[NT][KS][2];
-  float acc[NT][KS][4];
-  float m[NT][2];
-  float l[NT][2];
-  int lane;
-
-  __device__ __forceinline__ void init(const DecodeParams& p, int s, int hk, int lane_) {
-    lane = lane_;
-    const int r = lane >> 2, q4 = lane & 3;
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      const int g = nt * 8 + r;
-      const bool gv = g < p.group;
-      const void* qrow = static_cast<const uint16_t*>(p.q) + s * p.q_stride_s + (hk * p.group + (gv ? g : 0)) * p.q_stride_h;
-#pragma unroll
-      for (int ks = 0; ks < KS; ++ks) {
-        uint32_t b0 = 0, b1 = 0;
-        if (gv) {
-          if constexpr (C::kFp8) {
-            // Logical k (2q, 2q+1) <-> d = 16ks + 4q + {0,1}; (2q+8, 2q+9) <-> 16ks + 4q + {2,3}.
-            b0 = q_pair<C>(qrow, 16 * ks + 4 * q4);
-            b1 = q_pair<C>(qrow, 16 * ks + 4 * q4 + 2);
-          } else {
-            b0 = q_pair<C>(qrow, 16 * ks + 2 * q4);
-            b1 = q_pair<C>(qrow, 16 * ks + 2 * q4 + 8);
-          }
-        }
-        qf[nt][ks][0] = b0;
-        qf[nt][ks][1] = b1;
-      }
-#pragma unroll
-      for (int mt = 0; mt < KS; ++mt)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) acc[nt][mt][i] = 0.f;
-      m[nt][0] = m[nt][1] = -INFINITY;
-      l[nt][0] = l[nt][1] = 0.f;
-    }
-  }
-
-  // One 16-token page; kb/vb are the shared addresses of its K and V pages; nv valid tokens.
-  __device__ __forceinline__ void page(uint32_t kb, uint32_t vb, int nv, float sl2) {
-    const int x7 = lane & 7;
-    const int a_tok = (((lane >> 3) & 1) << 3) | x7;  // K (and e4m3 V) matrices: tok half = bit 3
-    const int a_co = lane >> 4;
-    const int t_tok = ((lane >> 4) << 3) | x7;        // 16-bit V^T matrices: tok half = bit 4
-    const int t_co = (lane >> 3) & 1;
-    const int r = lane >> 2, q4 = lane & 3;
-
-    // ---- S^T = K . Q^T --------------------------------------------------------------------
-    float sc[NT][4];
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
-    if constexpr (C::kFp8) {
-#pragma unroll
-      for (int kp = 0; kp < KS / 2; ++kp) {
-        uint32_t raw[4];
-        ldmatrix_x4(raw, kb + swz(a_tok, 2 * kp + a_co));
-        // a0a1 / a2a3 take codes (d 4q, 4q+1) of tokens r / r+8; a4a5 / a6a7 take (d 4q+2, 4q+3).
-        uint32_t a0[4], a1[4];
-        e4m3x4_to_f16x2x2(raw[0], a0[0], a0[2]);
-        e4m3x4_to_f16x2x2(raw[1], a0[1], a0[3]);
-        e4m3x4_to_f16x2x2(raw[2], a1[0], a1[2]);
-        e4m3x4_to_f16x2x2(raw[3], a1[1], a1[3]);
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          mma_16816<false>(sc[nt], a0, qf[nt][2 * kp][0], qf[nt][2 * kp][1]);
-          mma_16816<false>(sc[nt], a1, qf[nt][2 * kp + 1][0], qf[nt][2 * kp + 1][1]);
-        }
-      }
-    } else {
-#pragma unroll
-      for (int ks = 0; ks < KS; ++ks) {
-        uint32_t a[4];
-        ldmatrix_x4(a, kb + (ks >> 2) * 2048 + swz(a_tok, ((ks & 3) << 1) + a_co));
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) mma_16816<C::kMmaBf16>(sc[nt], a, qf[nt][ks][0], qf[nt][ks][1]);
-      }
-    }
-
-    // ---- online softmax over this page (log2 domain) -------------------------------------
-    const bool v_lo = r < nv, v_hi = r + 8 < nv;
-    uint32_t pf[NT][2];
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      float s0 = v_lo ? sc[nt][0] * sl2 : -INFINITY;
-      float s1 = v_lo ? sc[nt][1] * sl2 : -INFINITY;
-      float s2 = v_hi ? sc[nt][2] * sl2 : -INFINITY;
-      float s3 = v_hi ? sc[nt][3] * sl2 : -INFINITY;
-      float mx0 = fmaxf(s0, s2), mx1 = fmaxf(s1, s3);
-#pragma unroll
-      for (int off = 4; off < 32; off <<= 1) {
-        mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, off));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, off));
-      }
-      const float mn0 = fmaxf(m[nt][0], mx0), mn1 = fmaxf(m[nt][1], mx1);
-      const float al0 = ex2(m[nt][0] - mn0), al1 = ex2(m[nt][1] - mn1);
-      m[nt][0] = mn0;
-      m[nt][1] = mn1;
-      const uint32_t x0 = pack2<C::kMmaBf16>(ex2(s0 - mn0), ex2(s1 - mn1));
-      const uint32_t x1 = pack2<C::kMmaBf16>(ex2(s2 - mn0), ex2(s3 - mn1));
-      // The denominator sums the same rounded weights the PV product uses.
-      const float2 f0 = unpack2<C::kMmaBf16>(x0), f1 = unpack2<C::kMmaBf16>(x1);
-      l[nt][0] = l[nt][0] * al0 + (f0.x + f1.x);
-      l[nt][1] = l[nt][1] * al1 + (f0.y + f1.y);
-      if (__any_sync(kFull, al0 != 1.f || al1 != 1.f)) {  // skipped once the running max settles
-#pragma unroll
-        for (int mt = 0; mt < KS; ++mt) {
-          acc[nt][mt][0] *= al0;
-          acc[nt][mt][1] *= al1;
-          acc[nt][mt][2] *= al0;
-          acc[nt][mt][3] *= al1;
-        }
-      }
-      pf[nt][0] = movmatrix_trans(x0);  // (k = tok 2q, 2q+1 ; n = g = r)
-      pf[nt][1] = movmatrix_trans(x1);  // (k = tok 2q+8, 2q+9)
-    }
-
-    // Tokens past the context may hold any bits (NaN included): zero them in V^T so 0 * NaN
-    // never reaches the accumulator.
-    uint32_t mlo = 0xffffffffu, mhi = 0xffffffffu;
-    if (nv < 16) {
-      mlo = (2 * q4 < nv ? 0x0000ffffu : 0u) | (2 * q4 + 1 < nv ? 0xffff0000u : 0u);
-      mhi = (2 * q4 + 8 < nv ? 0x0000ffffu : 0u) | (2 * q4 + 9 < nv ? 0xffff0000u : 0u);
-    }
-
-    // ---- O^T += V^T . P^T -----------------------------------------------------------------
-    if constexpr (C::kFp8) {
-#pragma unroll
-      for (int mp = 0; mp < KS / 2; ++mp) {
-        uint32_t raw[4];
-        ldmatrix_x4_trans(raw, vb + swz(a_tok, 2 * mp + a_co));
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          // (tok 2q, d), (tok 2q, d+1), (tok 2q+1, d), (tok 2q+1, d+1) -> pairs of tokens per d.
-          const uint32_t t0 = __byte_perm(raw[2 * half], 0, 0x3120);
-          const uint32_t t1 = __byte_perm(raw[2 * half + 1], 0, 0x3120);
-          uint32_t a[4];
-          e4m3x4_to_f16x2x2(t0, a[0], a[1]);
-          e4m3x4_to_f16x2x2(t1, a[2], a[3]);
-          if (nv < 16) {
-            a[0] &= mlo;
-            a[1] &= mlo;
-            a[2] &= mhi;
-            a[3] &= mhi;
-          }
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt) mma_16816<false>(acc[nt][2 * mp + half], a, pf[nt][0], pf[nt][1]);
-        }
-      }
-    } else {
-#pragma unroll
-      for (int mt = 0; mt < KS; ++mt) {
-        uint32_t a[4];
-        ldmatrix_x4_trans(a, vb + (mt >> 2) * 2048 + swz(t_tok, ((mt & 3) << 1) + t_co));
-        if (nv < 16) {
-          a[0] &= mlo;
-          a[1] &= mlo;
-          a[2] &= mhi;
-          a[3] &= mhi;
-        }
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) mma_16816<C::kMmaBf16>(acc[nt][mt], a, pf[nt][0], pf[nt][1]);
-      }
-    }
-  }
-
-  // Write this warp's (m, l, acc) into the merge area: mg[g], lg[g], ag[g][D] (floats).
-  __device__ __forceinline__ void store(float* mg, float* lg, float* ag) {
-    const int r = lane >> 2, q4 = lane & 3;
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-#pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        float lv = l[nt][j];
-        lv += __shfl_xor_sync(kFull, lv, 4);
-        lv += __shfl_xor_sync(kFull, lv, 8);
-        lv += __shfl_xor_sync(kFull, lv, 16);
-        if (r == 0) {
-          mg[nt * 8 + 2 * q4 + j] = m[nt][j];
-          lg[nt * 8 + 2 * q4 + j] = lv;
-        }
-      }
-#pragma unroll
-      for (int mt = 0; mt < KS; ++mt) {
-        int d_lo, d_hi;
-        if constexpr (C::kFp8) {
-          d_lo = 16 * mt + 2 * r;
-          d_hi = d_lo + 1;
-        } else {
-          d_lo = 16 * mt + r;
-          d_hi = d_lo + 8;
-        }
-        const int g = nt * 8 + 2 * q4;
-        ag[g * D + d_lo] = acc[nt][mt][0];
-        ag[(g + 1) * D + d_lo] = acc[nt][mt][1];
-        ag[g * D + d_hi] = acc[nt][mt][2];
-        ag[(g + 1) * D + d_hi] = acc[nt][mt][3];
-      }
-    }
-  }
-};
 
 // ---------------------------------------------------------------------------------------------
 // CUDA-core per-page math (float32 FMA). Score phase: lane = (token t = lane & 15, half = lane >> 4),
@@ -847,19 +594,28 @@ __global__ void __launch_bounds__(Cfg<KV, QT, D, NT, KIND, OCC>::kThreads, Cfg<K
   }
 }
 
-// Merge the partitions of each (sequence, query head). blockDim.x / D groups (1 .. kReduceSplit) of D
-// threads take partitions k = w, w + groups, ... (eight per round, all of a round's loads in flight),
-// each keeping a running (M, num, den); the groups are then combined in fixed order, so the result is
-// deterministic. Many partitions get several groups; a handful get one.
-constexpr int kReduceSplit = 4;
+// Merge the partitions of each (sequence, query head): one CTA per row, one thread per d. A row's
+// partials are contiguous in the workspace, so they stream into shared memory as 1-D bulk copies of
+// kRedChunk partitions (kRedStages in flight); each thread keeps a running (M, num, den) over the
+// chunks in partition order, so the result is deterministic and independent of timing. The copies
+// keep the loads in flight without any thread waiting on them one by one.
+constexpr int kRedChunk = 16;
+constexpr int kRedStages = 4;
+constexpr int kRedMlBytes = kRedChunk * 8 + 16;  // a chunk's (m, l) pairs, copied from a 16-byte boundary
+template <int D>
+constexpr int reduce_smem_bytes() {
+  return kRedStages * (kRedChunk * D * 4 + kRedMlBytes) + kRedStages * 8;
+}
 template <int D, bool kBf16>
-__global__ void __launch_bounds__(kReduceSplit * D) reduce_kernel(const DecodeParams p) {
-  const int h = blockIdx.x, s = blockIdx.y, d = threadIdx.x % D, w = threadIdx.x / D;
-  const int groups = blockDim.x / D;
-  __shared__ float sm_num[kReduceSplit][D];
-  __shared__ float sm_m[kReduceSplit], sm_den[kReduceSplit];
+__global__ void __launch_bounds__(D) reduce_kernel(const DecodeParams p) {
+  extern __shared__ __align__(128) uint8_t red_smem[];
+  float* acc_s = reinterpret_cast<float*>(red_smem);                   // [stage][chunk][D]
+  uint8_t* ml_s = red_smem + kRedStages * kRedChunk * D * 4;            // [stage][kRedMlBytes]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ml_s + kRedStages * kRedMlBytes);
+  const int h = blockIdx.x, s = blockIdx.y, d = threadIdx.x;
+  // The next kernel on the stream is let in only as this grid's CTAs finish: a persistent decode grid
+  // after it should find the SMs free, not partly held by this merge.
   pdl_wait();  // the partials come from the decode grid just before this one
-  pdl_launch_dependents();
   const int Hq = p.num_kv_heads * p.group;
   const int PT = p.partition_tokens;
   const int ctx_cap = min(p.context_lens[s], p.max_blocks * 16);
@@ -867,51 +623,83 @@ __global__ void __launch_bounds__(kReduceSplit * D) reduce_kernel(const DecodePa
   const int np = p.part_offset + (span + PT - 1) / PT;
   if (!p.always_partials && np <= 1) return;  // the decode kernel wrote this row
   const int64_t row0 = (static_cast<int64_t>(s) * Hq + h) * p.ws_parts;
+  const int nchunks = (np + kRedChunk - 1) / kRedChunk;
+  const uint32_t bar0 = smem_u32(bars);
+  if (d == 0) {
+    for (int st = 0; st < kRedStages; ++st) mbar_init(bar0 + 8 * st, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  // Chunk i -> stage i % kRedStages, both copies started by thread 0: the acc rows, and the (m, l)
+  // pairs from the 16-byte boundary at or below their start (at most 8 bytes either side of the
+  // chunk's pairs, inside the workspace: its (m, l) area is a whole number of 256-byte lines).
+  auto ml_start = [&](int k0) { return (row0 + k0) * 8 & ~int64_t(15); };
+  auto issue = [&](int i) {
+    const int st = i % kRedStages, k0 = i * kRedChunk, n = min(kRedChunk, np - k0);
+    if (d == 0) {
+      const uint32_t acc_bytes = static_cast<uint32_t>(n) * D * 4;
+      const int64_t b0 = ml_start(k0), b1 = ((row0 + k0 + n) * 8 + 15) & ~int64_t(15);
+      const uint32_t ml_bytes = static_cast<uint32_t>(b1 - b0);
+      mbar_arrive_expect_tx(bar0 + 8 * st, acc_bytes + ml_bytes);
+      bulk_load_1d(smem_u32(acc_s + st * kRedChunk * D), p.ws_acc + (row0 + k0) * D, acc_bytes, bar0 + 8 * st);
+      bulk_load_1d(smem_u32(ml_s + st * kRedMlBytes), reinterpret_cast<const uint8_t*>(p.ws_ml) + b0, ml_bytes,
+                   bar0 + 8 * st);
+    }
+  };
+  for (int i = 0; i < min(kRedStages, nchunks); ++i) issue(i);
+  const uint64_t deadline = globaltimer_ns() + 2000000000ull;
   float M = -INFINITY, num = 0.f, den = 0.f;
-  for (int k0 = w; k0 < np; k0 += 8 * groups) {
-    float mk[8], lk[8], ak[8];
+  bool ok = true;
+  int i = 0;
+  for (; i < nchunks; ++i) {
+    const int st = i % kRedStages, n = min(kRedChunk, np - i * kRedChunk);
+    if (!__syncthreads_and(mbar_wait_bounded_poll(bar0 + 8 * st, (i / kRedStages) & 1, deadline))) {
+      ok = false;
+      break;
+    }
+    const int k0 = i * kRedChunk;
+    const float2* ml = reinterpret_cast<const float2*>(ml_s + st * kRedMlBytes + ((row0 + k0) * 8 - ml_start(k0)));
+    const float* a = acc_s + st * kRedChunk * D;
+    // Fully unrolled over the chunk (slots past n hold stale bytes: weight 0, values taken as 0), so
+    // the shared-memory loads and exponentials of all kRedChunk partitions overlap.
+    float mk[kRedChunk], lk[kRedChunk], ak[kRedChunk];
 #pragma unroll
-    for (int v = 0; v < 8; ++v) {
-      const int k = k0 + v * groups;
-      const int64_t slot = row0 + min(k, np - 1);
-      const float2 ml = *reinterpret_cast<const float2*>(p.ws_ml + slot * 2);
-      mk[v] = k < np ? ml.x : -INFINITY;
-      lk[v] = ml.y;
-      ak[v] = p.ws_acc[slot * D + d];
+    for (int k = 0; k < kRedChunk; ++k) {
+      const float2 v = ml[k];
+      mk[k] = k < n ? v.x : -INFINITY;
+      lk[k] = k < n ? v.y : 0.f;
+      ak[k] = k < n ? a[k * D + d] : 0.f;
     }
     float Mn = M;
 #pragma unroll
-    for (int v = 0; v < 8; ++v) Mn = fmaxf(Mn, mk[v]);
-    if (Mn == -INFINITY) continue;
-    const float a = ex2(M - Mn);
-    num *= a;
-    den *= a;
+    for (int k = 0; k < kRedChunk; ++k) Mn = fmaxf(Mn, mk[k]);
+    if (Mn != -INFINITY) {
+      const float r = ex2(M - Mn);
+      num *= r;
+      den *= r;
 #pragma unroll
-    for (int v = 0; v < 8; ++v) {
-      const float f = ex2(mk[v] - Mn);
-      num = fmaf(f, ak[v], num);
-      den = fmaf(f, lk[v], den);
+      for (int k = 0; k < kRedChunk; ++k) {
+        const float f = ex2(mk[k] - Mn);  // a partition without tokens has m = -inf: weight 0
+        num = fmaf(f, ak[k], num);
+        den = fmaf(f, lk[k], den);
+      }
+      M = Mn;
     }
-    M = Mn;
+    __syncthreads();  // every thread is done with this stage before it is refilled
+    if (i + kRedStages < nchunks) issue(i + kRedStages);
   }
-  sm_num[w][d] = num;
-  if (d == 0) {
-    sm_m[w] = M;
-    sm_den[w] = den;
+  if (!ok) {
+    // Let the copies still in flight land (bounded) before the CTA's shared memory goes.
+    if (d == 0) {
+      for (int k = i; k < min(i + kRedStages, nchunks); ++k)
+        mbar_wait_bounded(bar0 + 8 * (k % kRedStages), (k / kRedStages) & 1, globaltimer_ns() + 100000000ull);
+      atomicOr(p.err, 4u);
+    }
+    return;
   }
-  __syncthreads();
-  if (w != 0) return;
-  float Mt = -INFINITY;
-  for (int g = 0; g < groups; ++g) Mt = fmaxf(Mt, sm_m[g]);
   uint16_t bits = 0;  // no token at all (empty context): 0
-  if (Mt != -INFINITY) {
-    float nt = 0.f, dt = 0.f;
-    for (int g = 0; g < groups; ++g) {
-      const float f = ex2(sm_m[g] - Mt);  // a group without partitions has m = -inf: weight 0
-      nt = fmaf(f, sm_num[g][d], nt);
-      dt = fmaf(f, sm_den[g], dt);
-    }
-    const float o = nt / dt * p.v_scale;
+  if (M != -INFINITY) {
+    const float o = num / den * p.v_scale;
     if constexpr (kBf16) {
       bits = __bfloat16_as_ushort(__float2bfloat16_rn(o));
     } else {
@@ -919,23 +707,7 @@ __global__ void __launch_bounds__(kReduceSplit * D) reduce_kernel(const DecodePa
     }
   }
   static_cast<uint16_t*>(p.out)[s * p.o_stride_s + h * p.o_stride_h + d] = bits;
-}
-
-// Launch with programmatic stream serialisation: the kernel may begin while the previous kernel on
-// the stream finishes; it waits for it in pdl_wait() before reading anything.
-template <typename... KArgs, typename... Args>
-cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args&&... args) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = grid;
-  cfg.blockDim = block;
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+  pdl_launch_dependents();
 }
 
 template <KvType KV, QType QT, int D, int NT, int KIND, int OCC>
@@ -1008,15 +780,19 @@ cudaError_t launch_decode(const DecodeConfig& c, const CUtensorMap& km, const CU
                             : launch_kind<KvType::E4M3, QType::F16, 128>(c, g, km, vm, p, st);
 }
 
+template <int D, bool kBf16>
+cudaError_t launch_reduce_one(dim3 grid, const DecodeParams& p, cudaStream_t st) {
+  auto kern = reduce_kernel<D, kBf16>;
+  constexpr int smem = reduce_smem_bytes<D>();
+  static_assert(smem <= 48 * 1024, "no opt-in shared memory needed");
+  return launch_pdl(kern, grid, dim3(D), smem, st, p);
+}
+
 cudaError_t launch_reduce(const DecodeConfig& c, const DecodeParams& p, cudaStream_t st) {
   const dim3 grid(p.num_kv_heads * p.group, p.num_seqs);
   const bool bf = c.q == QType::BF16;
-  const unsigned groups = p.ws_parts > 8 ? kReduceSplit : 1;
-  if (c.head_dim == 128)
-    return bf ? launch_pdl(reduce_kernel<128, true>, grid, dim3(groups * 128), 0, st, p)
-              : launch_pdl(reduce_kernel<128, false>, grid, dim3(groups * 128), 0, st, p);
-  return bf ? launch_pdl(reduce_kernel<64, true>, grid, dim3(groups * 64), 0, st, p)
-            : launch_pdl(reduce_kernel<64, false>, grid, dim3(groups * 64), 0, st, p);
+  if (c.head_dim == 128) return bf ? launch_reduce_one<128, true>(grid, p, st) : launch_reduce_one<128, false>(grid, p, st);
+  return bf ? launch_reduce_one<64, true>(grid, p, st) : launch_reduce_one<64, false>(grid, p, st);
 }
 
 uint32_t* decode_error_word() {

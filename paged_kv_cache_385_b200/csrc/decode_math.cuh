@@ -1,0 +1,349 @@
+// Per-page tensor-core math and launch helpers shared by the decode kernels (decode.cu: one CTA per
+// (partition, KV head, sequence); decode_units.cu: one warp per partition, persistent).
+#pragma once
+
+#include <utility>
+
+#include "internal.h"
+#include "pa_device.cuh"
+
+namespace pa {
+
+// OCC is the number of CTAs per SM a kernel is compiled for: the page pipeline gets 192 KB / OCC of
+// shared memory (96, 64 or 48 KB) and registers are capped to fit. 16-bit pages with one query per
+// KV head are pure bandwidth: deep pipelines, 2 CTAs/SM. Grouped queries add math per byte and
+// e4m3 pages even more (widening, 3x the pages per byte moved), so those trade stages for resident
+// warps: 3 and 4 CTAs/SM.
+template <KvType KV, QType QT, int D, int NT, int KIND, int OCC>
+struct Cfg {
+  static constexpr bool kFp8 = KV == KvType::E4M3;
+  static constexpr int kEsz = kFp8 ? 1 : 2;
+  static constexpr int kRowBytes = D * kEsz;         // one token row of a page
+  static constexpr int kSubPages = kRowBytes / 128;  // 128-byte swizzled sub-pages per page
+  static constexpr int kSubElems = 128 / kEsz;       // TMA box width in elements
+  static constexpr int kPageBytes = 16 * kRowBytes;
+  static constexpr int kWarps = kDecodeWarps;
+  static constexpr int kThreads = kWarps * 32;
+  static constexpr int kStageBytes = 2 * kPageBytes;  // K page + V page
+  static constexpr int kMinBlocks = OCC;
+  static constexpr int kPipeBudget = OCC == 2 ? 96 * 1024 : (OCC == 3 ? 64 * 1024 : 48 * 1024);
+  static constexpr int kStages = kPipeBudget / (kWarps * kStageBytes);
+  static constexpr int kPipeBytes = kWarps * kStages * kStageBytes;
+  static constexpr bool kMmaBf16 = KV == KvType::BF16;  // e4m3 pages are widened to f16
+  static constexpr bool kQBf16 = QT == QType::BF16;
+  static constexpr int kGPad = 8 * NT;
+  static constexpr int kMergeFloats = kWarps * kGPad * (D + 2);
+  static constexpr int kSmemBytes = 1024 + kPipeBytes + kWarps * kStages * 8;
+  static_assert(kSubPages >= 1 && kRowBytes % 128 == 0, "page rows must be whole 128-byte lines");
+  static_assert(kStages >= 2, "need at least two stages per warp");
+  static_assert(kMergeFloats * 4 <= kPipeBytes, "merge area must fit in the pipeline buffers");
+};
+
+// Byte offset of 16-byte chunk `chunk` of token row `tok` in a 128-byte-swizzled sub-page.
+__device__ __forceinline__ uint32_t swz(int tok, int chunk) {
+  return static_cast<uint32_t>(tok * 128 + ((chunk ^ (tok & 7)) << 4));
+}
+
+template <class C>
+__device__ __forceinline__ uint32_t q_pair(const void* qrow, int d) {
+  // Two consecutive query elements (d, d+1) as the mma operand type.
+  const uint32_t raw = *reinterpret_cast<const uint32_t*>(static_cast<const uint16_t*>(qrow) + d);
+  if constexpr (C::kFp8 && C::kQBf16) {
+    const float2 f = unpack2<true>(raw);
+    return pack2<false>(f.x, f.y);
+  } else {
+    return raw;
+  }
+}
+
+// ---------------------------------------------------------------------------------------------
+// Tensor-core per-page math.
+// ---------------------------------------------------------------------------------------------
+template <class C, int D, int NT>
+struct TcMath {
+  static constexpr int KS = D / 16;  // k-steps of QK^T == m-tiles of PV
+  uint32_t qf[NT][KS][2];
+  float acc[NT][KS][4];
+  float m[NT][2];
+  float l[NT][2];
+  int lane;
+
+  __device__ __forceinline__ void init(const DecodeParams& p, int s, int hk, int lane_) {
+    lane = lane_;
+    const int r = lane >> 2, q4 = lane & 3;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const int g = nt * 8 + r;
+      const bool gv = g < p.group;
+      const void* qrow = static_cast<const uint16_t*>(p.q) + s * p.q_stride_s + (hk * p.group + (gv ? g : 0)) * p.q_stride_h;
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks) {
+        uint32_t b0 = 0, b1 = 0;
+        if (gv) {
+          if constexpr (C::kFp8) {
+            // Logical k (2q, 2q+1) <-> d = 16ks + 4q + {0,1}; (2q+8, 2q+9) <-> 16ks + 4q + {2,3}.
+            b0 = q_pair<C>(qrow, 16 * ks + 4 * q4);
+            b1 = q_pair<C>(qrow, 16 * ks + 4 * q4 + 2);
+          } else {
+            b0 = q_pair<C>(qrow, 16 * ks + 2 * q4);
+            b1 = q_pair<C>(qrow, 16 * ks + 2 * q4 + 8);
+          }
+        }
+        qf[nt][ks][0] = b0;
+        qf[nt][ks][1] = b1;
+      }
+#pragma unroll
+      for (int mt = 0; mt < KS; ++mt)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[nt][mt][i] = 0.f;
+      m[nt][0] = m[nt][1] = -INFINITY;
+      l[nt][0] = l[nt][1] = 0.f;
+    }
+  }
+
+  // One 16-token page; kb/vb are the shared addresses of its K and V pages; nv valid tokens.
+  __device__ __forceinline__ void page(uint32_t kb, uint32_t vb, int nv, float sl2) {
+    const int x7 = lane & 7;
+    const int a_tok = (((lane >> 3) & 1) << 3) | x7;  // K (and e4m3 V) matrices: tok half = bit 3
+    const int a_co = lane >> 4;
+    const int t_tok = ((lane >> 4) << 3) | x7;        // 16-bit V^T matrices: tok half = bit 4
+    const int t_co = (lane >> 3) & 1;
+    const int r = lane >> 2, q4 = lane & 3;
+
+    // ---- S^T = K . Q^T --------------------------------------------------------------------
+    float sc[NT][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+    if constexpr (C::kFp8) {
+#pragma unroll
+      for (int kp = 0; kp < KS / 2; ++kp) {
+        uint32_t raw[4];
+        ldmatrix_x4(raw, kb + swz(a_tok, 2 * kp + a_co));
+        // a0a1 / a2a3 take codes (d 4q, 4q+1) of tokens r / r+8; a4a5 / a6a7 take (d 4q+2, 4q+3).
+        uint32_t a0[4], a1[4];
+        e4m3x4_to_f16x2x2(raw[0], a0[0], a0[2]);
+        e4m3x4_to_f16x2x2(raw[1], a0[1], a0[3]);
+        e4m3x4_to_f16x2x2(raw[2], a1[0], a1[2]);
+        e4m3x4_to_f16x2x2(raw[3], a1[1], a1[3]);
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          mma_16816<false>(sc[nt], a0, qf[nt][2 * kp][0], qf[nt][2 * kp][1]);
+          mma_16816<false>(sc[nt], a1, qf[nt][2 * kp + 1][0], qf[nt][2 * kp + 1][1]);
+        }
+      }
+    } else {
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks) {
+        uint32_t a[4];
+        ldmatrix_x4(a, kb + (ks >> 2) * 2048 + swz(a_tok, ((ks & 3) << 1) + a_co));
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) mma_16816<C::kMmaBf16>(sc[nt], a, qf[nt][ks][0], qf[nt][ks][1]);
+      }
+    }
+
+    // ---- online softmax over this page (log2 domain) -------------------------------------
+    const bool v_lo = r < nv, v_hi = r + 8 < nv;
+    uint32_t pf[NT][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      float s0 = v_lo ? sc[nt][0] * sl2 : -INFINITY;
+      float s1 = v_lo ? sc[nt][1] * sl2 : -INFINITY;
+      float s2 = v_hi ? sc[nt][2] * sl2 : -INFINITY;
+      float s3 = v_hi ? sc[nt][3] * sl2 : -INFINITY;
+      float mx0 = fmaxf(s0, s2), mx1 = fmaxf(s1, s3);
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) {
+        mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, off));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, off));
+      }
+      const float mn0 = fmaxf(m[nt][0], mx0), mn1 = fmaxf(m[nt][1], mx1);
+      const float al0 = ex2(m[nt][0] - mn0), al1 = ex2(m[nt][1] - mn1);
+      m[nt][0] = mn0;
+      m[nt][1] = mn1;
+      const uint32_t x0 = pack2<C::kMmaBf16>(ex2(s0 - mn0), ex2(s1 - mn1));
+      const uint32_t x1 = pack2<C::kMmaBf16>(ex2(s2 - mn0), ex2(s3 - mn1));
+      // The denominator sums the same rounded weights the PV product uses.
+      const float2 f0 = unpack2<C::kMmaBf16>(x0), f1 = unpack2<C::kMmaBf16>(x1);
+      l[nt][0] = l[nt][0] * al0 + (f0.x + f1.x);
+      l[nt][1] = l[nt][1] * al1 + (f0.y + f1.y);
+      if (__any_sync(kFull, al0 != 1.f || al1 != 1.f)) {  // skipped once the running max settles
+#pragma unroll
+        for (int mt = 0; mt < KS; ++mt) {
+          acc[nt][mt][0] *= al0;
+          acc[nt][mt][1] *= al1;
+          acc[nt][mt][2] *= al0;
+          acc[nt][mt][3] *= al1;
+        }
+      }
+      pf[nt][0] = movmatrix_trans(x0);  // (k = tok 2q, 2q+1 ; n = g = r)
+      pf[nt][1] = movmatrix_trans(x1);  // (k = tok 2q+8, 2q+9)
+    }
+
+    // Tokens past the context may hold any bits (NaN included): zero them in V^T so 0 * NaN
+    // never reaches the accumulator.
+    uint32_t mlo = 0xffffffffu, mhi = 0xffffffffu;
+    if (nv < 16) {
+      mlo = (2 * q4 < nv ? 0x0000ffffu : 0u) | (2 * q4 + 1 < nv ? 0xffff0000u : 0u);
+      mhi = (2 * q4 + 8 < nv ? 0x0000ffffu : 0u) | (2 * q4 + 9 < nv ? 0xffff0000u : 0u);
+    }
+
+    // ---- O^T += V^T . P^T -----------------------------------------------------------------
+    if constexpr (C::kFp8) {
+#pragma unroll
+      for (int mp = 0; mp < KS / 2; ++mp) {
+        uint32_t raw[4];
+        ldmatrix_x4_trans(raw, vb + swz(a_tok, 2 * mp + a_co));
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          // (tok 2q, d), (tok 2q, d+1), (tok 2q+1, d), (tok 2q+1, d+1) -> pairs of tokens per d.
+          const uint32_t t0 = __byte_perm(raw[2 * half], 0, 0x3120);
+          const uint32_t t1 = __byte_perm(raw[2 * half + 1], 0, 0x3120);
+          uint32_t a[4];
+          e4m3x4_to_f16x2x2(t0, a[0], a[1]);
+          e4m3x4_to_f16x2x2(t1, a[2], a[3]);
+          if (nv < 16) {
+            a[0] &= mlo;
+            a[1] &= mlo;
+            a[2] &= mhi;
+            a[3] &= mhi;
+          }
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) mma_16816<false>(acc[nt][2 * mp + half], a, pf[nt][0], pf[nt][1]);
+        }
+      }
+    } else {
+#pragma unroll
+      for (int mt = 0; mt < KS; ++mt) {
+        uint32_t a[4];
+        ldmatrix_x4_trans(a, vb + (mt >> 2) * 2048 + swz(t_tok, ((mt & 3) << 1) + t_co));
+        if (nv < 16) {
+          a[0] &= mlo;
+          a[1] &= mlo;
+          a[2] &= mhi;
+          a[3] &= mhi;
+        }
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) mma_16816<C::kMmaBf16>(acc[nt][mt], a, pf[nt][0], pf[nt][1]);
+      }
+    }
+  }
+
+  // Zero the running state (a new partition, same query).
+  __device__ __forceinline__ void reset() {
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+      for (int mt = 0; mt < KS; ++mt)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[nt][mt][i] = 0.f;
+      m[nt][0] = m[nt][1] = -INFINITY;
+      l[nt][0] = l[nt][1] = 0.f;
+    }
+  }
+
+  // This warp's state written straight to global memory for query heads hk * G + g, g < G: with
+  // `direct`, the normalised output (acc / l * v_scale, rounded to nearest even; 0 when l is 0)
+  // into out; otherwise the partial (acc, m, l) into workspace slot `part` of each head's row, stored
+  // with L2 policy `keep` (the merge kernel reads it back right after).
+  template <bool kOutBf16>
+  __device__ __forceinline__ void write_global(const DecodeParams& p, int s, int hk, int part, bool direct,
+                                               uint64_t keep) {
+    const int r = lane >> 2, q4 = lane & 3;
+    const int G = p.group, Hq = p.num_kv_heads * G;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        float lv = l[nt][j];
+        lv += __shfl_xor_sync(kFull, lv, 4);
+        lv += __shfl_xor_sync(kFull, lv, 8);
+        lv += __shfl_xor_sync(kFull, lv, 16);
+        const int g = nt * 8 + 2 * q4 + j;
+        if (g >= G) continue;
+        const int h = hk * G + g;
+        if (direct) {
+          const float inv = lv > 0.f ? p.v_scale / lv : 0.f;
+          uint16_t* o = static_cast<uint16_t*>(p.out) + s * p.o_stride_s + h * p.o_stride_h;
+#pragma unroll
+          for (int mt = 0; mt < KS; ++mt) {
+            const float lo = acc[nt][mt][j] * inv, hi = acc[nt][mt][j + 2] * inv;
+            if constexpr (C::kFp8) {  // d = 16 mt + 2 r and the next one: one 32-bit store
+              *reinterpret_cast<uint32_t*>(o + 16 * mt + 2 * r) = pack2<kOutBf16>(lo, hi);
+            } else {  // d = 16 mt + r and 16 mt + r + 8
+              const uint32_t w = pack2<kOutBf16>(lo, hi);
+              o[16 * mt + r] = static_cast<uint16_t>(w & 0xffffu);
+              o[16 * mt + r + 8] = static_cast<uint16_t>(w >> 16);
+            }
+          }
+        } else {
+          const int64_t row = (static_cast<int64_t>(s) * Hq + h) * p.ws_parts + p.part_offset + part;
+          float* a = p.ws_acc + row * D;
+#pragma unroll
+          for (int mt = 0; mt < KS; ++mt) {
+            if constexpr (C::kFp8) {
+              st_global_hint(a + 16 * mt + 2 * r, make_float2(acc[nt][mt][j], acc[nt][mt][j + 2]), keep);
+            } else {
+              st_global_hint(a + 16 * mt + r, acc[nt][mt][j], keep);
+              st_global_hint(a + 16 * mt + r + 8, acc[nt][mt][j + 2], keep);
+            }
+          }
+          if (r == 0) st_global_hint(p.ws_ml + row * 2, make_float2(m[nt][j], lv), keep);
+        }
+      }
+    }
+  }
+
+  // Write this warp's (m, l, acc) into the merge area: mg[g], lg[g], ag[g][D] (floats).
+  __device__ __forceinline__ void store(float* mg, float* lg, float* ag) {
+    const int r = lane >> 2, q4 = lane & 3;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        float lv = l[nt][j];
+        lv += __shfl_xor_sync(kFull, lv, 4);
+        lv += __shfl_xor_sync(kFull, lv, 8);
+        lv += __shfl_xor_sync(kFull, lv, 16);
+        if (r == 0) {
+          mg[nt * 8 + 2 * q4 + j] = m[nt][j];
+          lg[nt * 8 + 2 * q4 + j] = lv;
+        }
+      }
+#pragma unroll
+      for (int mt = 0; mt < KS; ++mt) {
+        int d_lo, d_hi;
+        if constexpr (C::kFp8) {
+          d_lo = 16 * mt + 2 * r;
+          d_hi = d_lo + 1;
+        } else {
+          d_lo = 16 * mt + r;
+          d_hi = d_lo + 8;
+        }
+        const int g = nt * 8 + 2 * q4;
+        ag[g * D + d_lo] = acc[nt][mt][0];
+        ag[(g + 1) * D + d_lo] = acc[nt][mt][1];
+        ag[g * D + d_hi] = acc[nt][mt][2];
+        ag[(g + 1) * D + d_hi] = acc[nt][mt][3];
+      }
+    }
+  }
+};
+
+// Launch with programmatic stream serialisation: the kernel may begin while the previous kernel on
+// the stream finishes; it waits for it in pdl_wait() before reading anything.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
+}  // namespace pa

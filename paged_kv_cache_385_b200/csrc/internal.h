@@ -71,6 +71,15 @@ constexpr int kMaxPartitionTokens = 16 * 32 * kDecodeWarps;
 
 cudaError_t launch_decode(const DecodeConfig& cfg, const CUtensorMap& k_map, const CUtensorMap& v_map,
                           const DecodeParams& p, cudaStream_t stream);
+// Split decode with one persistent warp per partition (decode_units.cu): tensor-core kernel,
+// partitions of at most kUnitMaxPartitionTokens tokens (one page per lane), at most kUnitMaxSeqs
+// sequences (their unit counts live in shared memory), plain decode or pa_decode_step (not the
+// cascade suffix). Followed by launch_reduce like the per-partition CTAs.
+constexpr int kUnitMaxSeqs = 512;
+constexpr int kUnitMaxPartitionTokens = 512;
+bool decode_units_supported(const DecodeConfig& cfg, const DecodeParams& p);
+cudaError_t launch_decode_units(const DecodeConfig& cfg, const CUtensorMap& k_map, const CUtensorMap& v_map,
+                                const DecodeParams& p, cudaStream_t stream);
 cudaError_t launch_reduce(const DecodeConfig& cfg, const DecodeParams& p, cudaStream_t stream);
 bool decode_supported(const DecodeConfig& cfg);
 

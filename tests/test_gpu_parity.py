@@ -52,7 +52,9 @@ def test_pool_bytes_bit_exact(name):
 
 
 def _kernels(w):
-    return [1, 0] if w.group <= 8 else [1]
+    """Tensor-core (split contexts: one persistent warp per partition), tensor-core with one CTA per
+    partition, and the CUDA-core kernel (query groups of at most 8)."""
+    return [1, 2, 0] if w.group <= 8 else [1, 2]
 
 
 @pytest.mark.parametrize("name", SMALL)
