@@ -594,29 +594,40 @@ __global__ void __launch_bounds__(Cfg<KV, QT, D, NT, KIND, OCC>::kThreads, Cfg<K
   }
 }
 
-// Merge the partitions of each (sequence, query head): one CTA per row, one thread per d. A row's
+// Merge the partitions of each (sequence, query head): one CTA per row, kRedWarps warps. A row's
 // partials are contiguous in the workspace, so they stream into shared memory as 1-D bulk copies of
-// kRedChunk partitions (kRedStages in flight); each thread keeps a running (M, num, den) over the
-// chunks in partition order, so the result is deterministic and independent of timing. The copies
-// keep the loads in flight without any thread waiting on them one by one.
+// kRedChunk partitions (acc rows, and the (m, l) pairs from the 16-byte boundary at or below their
+// start); chunk c goes to warp c % kRedWarps, each warp with kRedStages chunks in flight. Lane k of a
+// chunk takes partition k's (m, l): the chunk's maximum and weights come from warp shuffles, and each
+// lane accumulates its D / 32 values of d over the chunk's partitions in order. The warps' states are
+// then combined in warp order. Every order is fixed, so the result is deterministic.
 constexpr int kRedChunk = 16;
 constexpr int kRedStages = 4;
-constexpr int kRedMlBytes = kRedChunk * 8 + 16;  // a chunk's (m, l) pairs, copied from a 16-byte boundary
+constexpr int kRedWarps = 2;
+constexpr int kRedMlBytes = kRedChunk * 8 + 16;
 template <int D>
-constexpr int reduce_smem_bytes() {
-  return kRedStages * (kRedChunk * D * 4 + kRedMlBytes) + kRedStages * 8;
-}
+struct RedCfg {
+  static constexpr int kAccBytes = kRedChunk * D * 4;  // one chunk of acc rows
+  static constexpr int kWarpBytes = kRedStages * (kAccBytes + kRedMlBytes + 8);
+  static constexpr int kCombineBytes = kRedWarps * (D + 2) * 4;
+  static constexpr int kSmemBytes = kRedWarps * kWarpBytes + kCombineBytes;
+};
 template <int D, bool kBf16>
-__global__ void __launch_bounds__(D) reduce_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__(kRedWarps * 32) reduce_kernel(const DecodeParams p) {
+  using R = RedCfg<D>;
+  constexpr int V = D / 32;  // values of d per lane
   extern __shared__ __align__(128) uint8_t red_smem[];
-  float* acc_s = reinterpret_cast<float*>(red_smem);                   // [stage][chunk][D]
-  uint8_t* ml_s = red_smem + kRedStages * kRedChunk * D * 4;            // [stage][kRedMlBytes]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(ml_s + kRedStages * kRedMlBytes);
-  const int h = blockIdx.x, s = blockIdx.y, d = threadIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint8_t* wsm = red_smem + warp * R::kWarpBytes;
+  float* acc_s = reinterpret_cast<float*>(wsm);                       // [stage][chunk][D]
+  uint8_t* ml_s = wsm + kRedStages * R::kAccBytes;                     // [stage][kRedMlBytes]
+  const uint32_t bar0 = smem_u32(ml_s + kRedStages * kRedMlBytes);     // [stage]
+  float* comb = reinterpret_cast<float*>(red_smem + kRedWarps * R::kWarpBytes);  // [warp][D + 2]
   // The next kernel on the stream is let in only as this grid's CTAs finish: a persistent decode grid
   // after it should find the SMs free, not partly held by this merge.
   pdl_wait();  // the partials come from the decode grid just before this one
   const int Hq = p.num_kv_heads * p.group;
+  const int h = blockIdx.x, s = blockIdx.y;
   const int PT = p.partition_tokens;
   const int ctx_cap = min(p.context_lens[s], p.max_blocks * 16);
   const int span = min(max(ctx_cap - p.start_tokens, 0), p.num_partitions * PT);
@@ -624,89 +635,123 @@ __global__ void __launch_bounds__(D) reduce_kernel(const DecodeParams p) {
   if (!p.always_partials && np <= 1) return;  // the decode kernel wrote this row
   const int64_t row0 = (static_cast<int64_t>(s) * Hq + h) * p.ws_parts;
   const int nchunks = (np + kRedChunk - 1) / kRedChunk;
-  const uint32_t bar0 = smem_u32(bars);
-  if (d == 0) {
+  const int mine_n = nchunks > warp ? (nchunks - warp + kRedWarps - 1) / kRedWarps : 0;  // this warp's chunks
+  if (lane == 0) {
     for (int st = 0; st < kRedStages; ++st) mbar_init(bar0 + 8 * st, 1);
     fence_barrier_init();
   }
-  __syncthreads();
-  // Chunk i -> stage i % kRedStages, both copies started by thread 0: the acc rows, and the (m, l)
-  // pairs from the 16-byte boundary at or below their start (at most 8 bytes either side of the
-  // chunk's pairs, inside the workspace: its (m, l) area is a whole number of 256-byte lines).
+  __syncwarp();
+  // The warp's j-th chunk (chunk warp + j * kRedWarps) -> stage j % kRedStages. The (m, l) copy may
+  // take up to 8 bytes on either side of the chunk's pairs, still inside the workspace: its (m, l)
+  // area is a whole number of 256-byte lines.
   auto ml_start = [&](int k0) { return (row0 + k0) * 8 & ~int64_t(15); };
-  auto issue = [&](int i) {
-    const int st = i % kRedStages, k0 = i * kRedChunk, n = min(kRedChunk, np - k0);
-    if (d == 0) {
-      const uint32_t acc_bytes = static_cast<uint32_t>(n) * D * 4;
-      const int64_t b0 = ml_start(k0), b1 = ((row0 + k0 + n) * 8 + 15) & ~int64_t(15);
-      const uint32_t ml_bytes = static_cast<uint32_t>(b1 - b0);
-      mbar_arrive_expect_tx(bar0 + 8 * st, acc_bytes + ml_bytes);
-      bulk_load_1d(smem_u32(acc_s + st * kRedChunk * D), p.ws_acc + (row0 + k0) * D, acc_bytes, bar0 + 8 * st);
-      bulk_load_1d(smem_u32(ml_s + st * kRedMlBytes), reinterpret_cast<const uint8_t*>(p.ws_ml) + b0, ml_bytes,
-                   bar0 + 8 * st);
-    }
+  auto issue = [&](int j) {
+    if (lane != 0) return;
+    const int st = j % kRedStages, k0 = (warp + j * kRedWarps) * kRedChunk, n = min(kRedChunk, np - k0);
+    const uint32_t acc_bytes = static_cast<uint32_t>(n) * D * 4;
+    const int64_t b0 = ml_start(k0), b1 = ((row0 + k0 + n) * 8 + 15) & ~int64_t(15);
+    const uint32_t ml_bytes = static_cast<uint32_t>(b1 - b0);
+    mbar_arrive_expect_tx(bar0 + 8 * st, acc_bytes + ml_bytes);
+    bulk_load_1d(smem_u32(acc_s + st * kRedChunk * D), p.ws_acc + (row0 + k0) * D, acc_bytes, bar0 + 8 * st);
+    bulk_load_1d(smem_u32(ml_s + st * kRedMlBytes), reinterpret_cast<const uint8_t*>(p.ws_ml) + b0, ml_bytes,
+                 bar0 + 8 * st);
   };
-  for (int i = 0; i < min(kRedStages, nchunks); ++i) issue(i);
+  for (int j = 0; j < min(kRedStages, mine_n); ++j) issue(j);
   const uint64_t deadline = globaltimer_ns() + 2000000000ull;
-  float M = -INFINITY, num = 0.f, den = 0.f;
+  float M = -INFINITY, den = 0.f, num[V];
+#pragma unroll
+  for (int v = 0; v < V; ++v) num[v] = 0.f;
   bool ok = true;
-  int i = 0;
-  for (; i < nchunks; ++i) {
-    const int st = i % kRedStages, n = min(kRedChunk, np - i * kRedChunk);
-    if (!__syncthreads_and(mbar_wait_bounded_poll(bar0 + 8 * st, (i / kRedStages) & 1, deadline))) {
+  int j = 0;
+  for (; j < mine_n; ++j) {
+    const int st = j % kRedStages, k0 = (warp + j * kRedWarps) * kRedChunk, n = min(kRedChunk, np - k0);
+    if (!__all_sync(kFull, mbar_wait_bounded(bar0 + 8 * st, (j / kRedStages) & 1, deadline))) {
       ok = false;
       break;
     }
-    const int k0 = i * kRedChunk;
     const float2* ml = reinterpret_cast<const float2*>(ml_s + st * kRedMlBytes + ((row0 + k0) * 8 - ml_start(k0)));
     const float* a = acc_s + st * kRedChunk * D;
-    // Fully unrolled over the chunk (slots past n hold stale bytes: weight 0, values taken as 0), so
-    // the shared-memory loads and exponentials of all kRedChunk partitions overlap.
-    float mk[kRedChunk], lk[kRedChunk], ak[kRedChunk];
+    const float2 mine = lane < n ? ml[lane] : make_float2(-INFINITY, 0.f);
+    float cmax = mine.x;
 #pragma unroll
-    for (int k = 0; k < kRedChunk; ++k) {
-      const float2 v = ml[k];
-      mk[k] = k < n ? v.x : -INFINITY;
-      lk[k] = k < n ? v.y : 0.f;
-      ak[k] = k < n ? a[k * D + d] : 0.f;
-    }
-    float Mn = M;
-#pragma unroll
-    for (int k = 0; k < kRedChunk; ++k) Mn = fmaxf(Mn, mk[k]);
+    for (int off = 16; off > 0; off >>= 1) cmax = fmaxf(cmax, __shfl_xor_sync(kFull, cmax, off));
+    const float Mn = fmaxf(M, cmax);
     if (Mn != -INFINITY) {
       const float r = ex2(M - Mn);
-      num *= r;
-      den *= r;
+      const float f = ex2(mine.x - Mn);  // a partition without tokens has m = -inf: weight 0
+      float fl = f * mine.y;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) fl += __shfl_xor_sync(kFull, fl, off);
+      den = den * r + fl;
+#pragma unroll
+      for (int v = 0; v < V; ++v) num[v] *= r;
 #pragma unroll
       for (int k = 0; k < kRedChunk; ++k) {
-        const float f = ex2(mk[k] - Mn);  // a partition without tokens has m = -inf: weight 0
-        num = fmaf(f, ak[k], num);
-        den = fmaf(f, lk[k], den);
+        const float fk = __shfl_sync(kFull, f, k);
+        if (k < n) {  // slots past n hold stale bytes
+          if constexpr (V == 4) {
+            const float4 x = *reinterpret_cast<const float4*>(a + k * D + 4 * lane);
+            num[0] = fmaf(fk, x.x, num[0]);
+            num[1] = fmaf(fk, x.y, num[1]);
+            num[2] = fmaf(fk, x.z, num[2]);
+            num[3] = fmaf(fk, x.w, num[3]);
+          } else {
+            const float2 x = *reinterpret_cast<const float2*>(a + k * D + 2 * lane);
+            num[0] = fmaf(fk, x.x, num[0]);
+            num[1] = fmaf(fk, x.y, num[1]);
+          }
+        }
       }
       M = Mn;
     }
-    __syncthreads();  // every thread is done with this stage before it is refilled
-    if (i + kRedStages < nchunks) issue(i + kRedStages);
+    __syncwarp();  // every lane is done with this stage before it is refilled
+    if (j + kRedStages < mine_n) issue(j + kRedStages);
   }
   if (!ok) {
     // Let the copies still in flight land (bounded) before the CTA's shared memory goes.
-    if (d == 0) {
-      for (int k = i; k < min(i + kRedStages, nchunks); ++k)
+    if (lane == 0) {
+      for (int k = j; k < min(j + kRedStages, mine_n); ++k)
         mbar_wait_bounded(bar0 + 8 * (k % kRedStages), (k / kRedStages) & 1, globaltimer_ns() + 100000000ull);
       atomicOr(p.err, 4u);
     }
-    return;
   }
-  uint16_t bits = 0;  // no token at all (empty context): 0
-  if (M != -INFINITY) {
-    const float o = num / den * p.v_scale;
-    if constexpr (kBf16) {
-      bits = __bfloat16_as_ushort(__float2bfloat16_rn(o));
-    } else {
-      bits = __half_as_ushort(__float2half_rn(o));
+  // Combine the warps in warp order.
+  float* cw = comb + warp * (D + 2);
+#pragma unroll
+  for (int v = 0; v < V; ++v) cw[V * lane + v] = num[v];
+  if (lane == 0) {
+    cw[D] = M;
+    cw[D + 1] = den;
+  }
+  if (__syncthreads_or(!ok) || warp != 0) return;
+  float Mt = -INFINITY;
+#pragma unroll
+  for (int w = 0; w < kRedWarps; ++w) Mt = fmaxf(Mt, comb[w * (D + 2) + D]);
+  uint32_t out_w[V / 2];
+#pragma unroll
+  for (int v = 0; v < V / 2; ++v) out_w[v] = 0u;  // no token at all (empty context): 0
+  if (Mt != -INFINITY) {
+    float nt[V], dt = 0.f;
+#pragma unroll
+    for (int v = 0; v < V; ++v) nt[v] = 0.f;
+#pragma unroll
+    for (int w = 0; w < kRedWarps; ++w) {
+      const float* c = comb + w * (D + 2);
+      const float f = ex2(c[D] - Mt);  // a warp without partitions has m = -inf: weight 0
+      dt = fmaf(f, c[D + 1], dt);
+#pragma unroll
+      for (int v = 0; v < V; ++v) nt[v] = fmaf(f, c[V * lane + v], nt[v]);
     }
+    const float sc = p.v_scale / dt;
+#pragma unroll
+    for (int v = 0; v < V / 2; ++v) out_w[v] = pack2<kBf16>(nt[2 * v] * sc, nt[2 * v + 1] * sc);
   }
-  static_cast<uint16_t*>(p.out)[s * p.o_stride_s + h * p.o_stride_h + d] = bits;
+  uint16_t* o = static_cast<uint16_t*>(p.out) + s * p.o_stride_s + h * p.o_stride_h + V * lane;
+  if constexpr (V == 4) {
+    *reinterpret_cast<uint2*>(o) = make_uint2(out_w[0], out_w[1]);
+  } else {
+    *reinterpret_cast<uint32_t*>(o) = out_w[0];
+  }
   pdl_launch_dependents();
 }
 
@@ -781,18 +826,26 @@ cudaError_t launch_decode(const DecodeConfig& c, const CUtensorMap& km, const CU
 }
 
 template <int D, bool kBf16>
-cudaError_t launch_reduce_one(dim3 grid, const DecodeParams& p, cudaStream_t st) {
+cudaError_t launch_reduce_one(const DecodeParams& p, cudaStream_t st) {
   auto kern = reduce_kernel<D, kBf16>;
-  constexpr int smem = reduce_smem_bytes<D>();
-  static_assert(smem <= 48 * 1024, "no opt-in shared memory needed");
-  return launch_pdl(kern, grid, dim3(D), smem, st, p);
+  constexpr int smem = RedCfg<D>::kSmemBytes;
+  static int configured_devices = 0;  // bit per device
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 31 || !(__atomic_load_n(&configured_devices, __ATOMIC_ACQUIRE) & (1 << dev))) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    if (dev < 31) __atomic_fetch_or(&configured_devices, 1 << dev, __ATOMIC_ACQ_REL);
+  }
+  const dim3 grid(p.num_kv_heads * p.group, p.num_seqs);
+  return launch_pdl(kern, grid, dim3(kRedWarps * 32), smem, st, p);
 }
 
 cudaError_t launch_reduce(const DecodeConfig& c, const DecodeParams& p, cudaStream_t st) {
-  const dim3 grid(p.num_kv_heads * p.group, p.num_seqs);
   const bool bf = c.q == QType::BF16;
-  if (c.head_dim == 128) return bf ? launch_reduce_one<128, true>(grid, p, st) : launch_reduce_one<128, false>(grid, p, st);
-  return bf ? launch_reduce_one<64, true>(grid, p, st) : launch_reduce_one<64, false>(grid, p, st);
+  if (c.head_dim == 128) return bf ? launch_reduce_one<128, true>(p, st) : launch_reduce_one<128, false>(p, st);
+  return bf ? launch_reduce_one<64, true>(p, st) : launch_reduce_one<64, false>(p, st);
 }
 
 uint32_t* decode_error_word() {

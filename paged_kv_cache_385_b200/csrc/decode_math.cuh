@@ -101,10 +101,22 @@ struct TcMath {
     }
   }
 
+  // Token held in row m of S^T (and in k-slot m of the P.V product). 16-bit pages: m itself. e4m3
+  // pages: the order pi(m) = 4 (m' >> 1) + (m' & 1) + 2 (m >> 3), m' = m & 7, which puts tokens
+  // 4 q .. 4 q + 3 in the k-slots (2q, 2q+1, 2q+8, 2q+9) that lane q of the P.V product covers: the
+  // order a transposed byte ldmatrix delivers V in, so V needs no byte shuffles before widening.
+  static __device__ __forceinline__ int tok_of_row(int m) {
+    if constexpr (C::kFp8) {
+      return 4 * ((m & 7) >> 1) + (m & 1) + 2 * (m >> 3);
+    } else {
+      return m;
+    }
+  }
+
   // One 16-token page; kb/vb are the shared addresses of its K and V pages; nv valid tokens.
   __device__ __forceinline__ void page(uint32_t kb, uint32_t vb, int nv, float sl2) {
     const int x7 = lane & 7;
-    const int a_tok = (((lane >> 3) & 1) << 3) | x7;  // K (and e4m3 V) matrices: tok half = bit 3
+    const int a_tok = tok_of_row((((lane >> 3) & 1) << 3) | x7);  // K matrices: row half = bit 3
     const int a_co = lane >> 4;
     const int t_tok = ((lane >> 4) << 3) | x7;        // 16-bit V^T matrices: tok half = bit 4
     const int t_co = (lane >> 3) & 1;
@@ -142,7 +154,7 @@ struct TcMath {
     }
 
     // ---- online softmax over this page (log2 domain) -------------------------------------
-    const bool v_lo = r < nv, v_hi = r + 8 < nv;
+    const bool v_lo = tok_of_row(r) < nv, v_hi = tok_of_row(r + 8) < nv;
     uint32_t pf[NT][2];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
@@ -180,27 +192,28 @@ struct TcMath {
     }
 
     // Tokens past the context may hold any bits (NaN included): zero them in V^T so 0 * NaN
-    // never reaches the accumulator.
+    // never reaches the accumulator. mlo covers k-slots 2q, 2q+1, mhi k-slots 2q+8, 2q+9.
     uint32_t mlo = 0xffffffffu, mhi = 0xffffffffu;
     if (nv < 16) {
-      mlo = (2 * q4 < nv ? 0x0000ffffu : 0u) | (2 * q4 + 1 < nv ? 0xffff0000u : 0u);
-      mhi = (2 * q4 + 8 < nv ? 0x0000ffffu : 0u) | (2 * q4 + 9 < nv ? 0xffff0000u : 0u);
+      const int t0 = tok_of_row(2 * q4), t8 = tok_of_row(2 * q4 + 8);
+      mlo = (t0 < nv ? 0x0000ffffu : 0u) | (t0 + 1 < nv ? 0xffff0000u : 0u);
+      mhi = (t8 < nv ? 0x0000ffffu : 0u) | (t8 + 1 < nv ? 0xffff0000u : 0u);
     }
 
     // ---- O^T += V^T . P^T -----------------------------------------------------------------
     if constexpr (C::kFp8) {
+      // Lanes 0-15 address token rows of chunk 2 mp, lanes 16-31 those of chunk 2 mp + 1 (16 d each);
+      // each lane gets tokens 4 q .. 4 q + 3 of d = r and r + 8 of both chunks: k-slots (2q, 2q+1)
+      // and (2q+8, 2q+9) of m-tiles 2 mp and 2 mp + 1 after widening.
 #pragma unroll
       for (int mp = 0; mp < KS / 2; ++mp) {
         uint32_t raw[4];
-        ldmatrix_x4_trans(raw, vb + swz(a_tok, 2 * mp + a_co));
+        ldmatrix_b8_x2_trans(raw, vb + swz(lane & 15, 2 * mp + (lane >> 4)));
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
-          // (tok 2q, d), (tok 2q, d+1), (tok 2q+1, d), (tok 2q+1, d+1) -> pairs of tokens per d.
-          const uint32_t t0 = __byte_perm(raw[2 * half], 0, 0x3120);
-          const uint32_t t1 = __byte_perm(raw[2 * half + 1], 0, 0x3120);
           uint32_t a[4];
-          e4m3x4_to_f16x2x2(t0, a[0], a[1]);
-          e4m3x4_to_f16x2x2(t1, a[2], a[3]);
+          e4m3x4_to_f16x2x2(raw[2 * half], a[0], a[2]);
+          e4m3x4_to_f16x2x2(raw[2 * half + 1], a[1], a[3]);
           if (nv < 16) {
             a[0] &= mlo;
             a[1] &= mlo;
@@ -267,25 +280,17 @@ struct TcMath {
 #pragma unroll
           for (int mt = 0; mt < KS; ++mt) {
             const float lo = acc[nt][mt][j] * inv, hi = acc[nt][mt][j + 2] * inv;
-            if constexpr (C::kFp8) {  // d = 16 mt + 2 r and the next one: one 32-bit store
-              *reinterpret_cast<uint32_t*>(o + 16 * mt + 2 * r) = pack2<kOutBf16>(lo, hi);
-            } else {  // d = 16 mt + r and 16 mt + r + 8
-              const uint32_t w = pack2<kOutBf16>(lo, hi);
-              o[16 * mt + r] = static_cast<uint16_t>(w & 0xffffu);
-              o[16 * mt + r + 8] = static_cast<uint16_t>(w >> 16);
-            }
+            const uint32_t w = pack2<kOutBf16>(lo, hi);  // d = 16 mt + r and 16 mt + r + 8
+            o[16 * mt + r] = static_cast<uint16_t>(w & 0xffffu);
+            o[16 * mt + r + 8] = static_cast<uint16_t>(w >> 16);
           }
         } else {
           const int64_t row = (static_cast<int64_t>(s) * Hq + h) * p.ws_parts + p.part_offset + part;
           float* a = p.ws_acc + row * D;
 #pragma unroll
           for (int mt = 0; mt < KS; ++mt) {
-            if constexpr (C::kFp8) {
-              st_global_hint(a + 16 * mt + 2 * r, make_float2(acc[nt][mt][j], acc[nt][mt][j + 2]), keep);
-            } else {
-              st_global_hint(a + 16 * mt + r, acc[nt][mt][j], keep);
-              st_global_hint(a + 16 * mt + r + 8, acc[nt][mt][j + 2], keep);
-            }
+            st_global_hint(a + 16 * mt + r, acc[nt][mt][j], keep);
+            st_global_hint(a + 16 * mt + r + 8, acc[nt][mt][j + 2], keep);
           }
           if (r == 0) st_global_hint(p.ws_ml + row * 2, make_float2(m[nt][j], lv), keep);
         }
@@ -311,14 +316,7 @@ struct TcMath {
       }
 #pragma unroll
       for (int mt = 0; mt < KS; ++mt) {
-        int d_lo, d_hi;
-        if constexpr (C::kFp8) {
-          d_lo = 16 * mt + 2 * r;
-          d_hi = d_lo + 1;
-        } else {
-          d_lo = 16 * mt + r;
-          d_hi = d_lo + 8;
-        }
+        const int d_lo = 16 * mt + r, d_hi = d_lo + 8;
         const int g = nt * 8 + 2 * q4;
         ag[g * D + d_lo] = acc[nt][mt][0];
         ag[(g + 1) * D + d_lo] = acc[nt][mt][1];

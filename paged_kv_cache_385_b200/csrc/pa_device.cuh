@@ -172,6 +172,15 @@ __device__ __forceinline__ void ldmatrix_x4_trans(uint32_t (&r)[4], uint32_t add
                : "r"(addr));
 }
 
+// Two 16x16 byte matrices, transposed (sm_100a): lanes 0-15 give the row addresses of matrix 0 (16
+// bytes each), lanes 16-31 those of matrix 1. Lane L receives rows 4 (L & 3) .. 4 (L & 3) + 3 of column
+// L >> 2 (r[0]: matrix 0, r[2]: matrix 1) and of column (L >> 2) + 8 (r[1], r[3]), one row per byte.
+__device__ __forceinline__ void ldmatrix_b8_x2_trans(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m16n16.x2.trans.shared.b8 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
 // D = A(16x16, row) * B(16x8, col) + D with f32 accumulation; A/B both f16 or both bf16.
 template <bool kBf16>
 __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
