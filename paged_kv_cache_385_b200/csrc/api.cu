@@ -493,6 +493,9 @@ static int decode_impl(pa_tensor* out, const pa_tensor* q, const pa_tensor* k_ca
   p.always_partials = cascade ? 1 : 0;
   p.merge_prefix_inline = cascade && P == 1 ? 1 : 0;
   p.late_dependency_wait = cascade ? 1 : 0;
+  // The persistent per-warp split form where it applies (not the cascade suffix: its short units
+  // stream faster with a CTA's four warps on each); else one CTA per partition.
+  const bool use_units = ws_parts > 1 && !cta_per_partition && pa::decode_units_supported(cfg, p);
   size_t ml_off = 0;
   if (ws_parts > 1) {
     const size_t need = workspace_layout(B, Hq, D, ws_parts, &ml_off);
@@ -598,7 +601,7 @@ static int decode_impl(pa_tensor* out, const pa_tensor* q, const pa_tensor* k_ca
     }
     if (e != cudaSuccess) return fail(PA_ERR_CUDA, "prefix launch: %s", cudaGetErrorString(e));
   }
-  if (ws_parts > 1 && !cta_per_partition && pa::decode_units_supported(cfg, p))
+  if (use_units)
     e = pa::launch_decode_units(cfg, km, vm, p, s);
   else
     e = pa::launch_decode(cfg, km, vm, p, s);

@@ -594,27 +594,29 @@ __global__ void __launch_bounds__(Cfg<KV, QT, D, NT, KIND, OCC>::kThreads, Cfg<K
   }
 }
 
-// Merge the partitions of each (sequence, query head): one CTA per row, kRedWarps warps. A row's
+// Merge the partitions of each (sequence, query head): one CTA per row, W warps. A row's
 // partials are contiguous in the workspace, so they stream into shared memory as 1-D bulk copies of
 // kRedChunk partitions (acc rows, and the (m, l) pairs from the 16-byte boundary at or below their
-// start); chunk c goes to warp c % kRedWarps, each warp with kRedStages chunks in flight. Lane k of a
+// start); chunk c goes to warp c % W, each warp with S chunks in flight (fewer warps and stages for
+// short rows, so that many rows fit on an SM at once). Lane k of a
 // chunk takes partition k's (m, l): the chunk's maximum and weights come from warp shuffles, and each
 // lane accumulates its D / 32 values of d over the chunk's partitions in order. The warps' states are
 // then combined in warp order. Every order is fixed, so the result is deterministic.
 constexpr int kRedChunk = 16;
-constexpr int kRedStages = 4;
-constexpr int kRedWarps = 2;
 constexpr int kRedMlBytes = kRedChunk * 8 + 16;
-template <int D>
+template <int D, int W, int S>
 struct RedCfg {
+  static constexpr int kRedWarps = W;
+  static constexpr int kRedStages = S;
   static constexpr int kAccBytes = kRedChunk * D * 4;  // one chunk of acc rows
   static constexpr int kWarpBytes = kRedStages * (kAccBytes + kRedMlBytes + 8);
   static constexpr int kCombineBytes = kRedWarps * (D + 2) * 4;
   static constexpr int kSmemBytes = kRedWarps * kWarpBytes + kCombineBytes;
 };
-template <int D, bool kBf16>
-__global__ void __launch_bounds__(kRedWarps * 32) reduce_kernel(const DecodeParams p) {
-  using R = RedCfg<D>;
+template <int D, bool kBf16, int W, int S>
+__global__ void __launch_bounds__(W * 32) reduce_kernel(const DecodeParams p) {
+  using R = RedCfg<D, W, S>;
+  constexpr int kRedWarps = W, kRedStages = S;
   constexpr int V = D / 32;  // values of d per lane
   extern __shared__ __align__(128) uint8_t red_smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -825,10 +827,10 @@ cudaError_t launch_decode(const DecodeConfig& c, const CUtensorMap& km, const CU
                             : launch_kind<KvType::E4M3, QType::F16, 128>(c, g, km, vm, p, st);
 }
 
-template <int D, bool kBf16>
+template <int D, bool kBf16, int W, int S>
 cudaError_t launch_reduce_one(const DecodeParams& p, cudaStream_t st) {
-  auto kern = reduce_kernel<D, kBf16>;
-  constexpr int smem = RedCfg<D>::kSmemBytes;
+  auto kern = reduce_kernel<D, kBf16, W, S>;
+  constexpr int smem = RedCfg<D, W, S>::kSmemBytes;
   static int configured_devices = 0;  // bit per device
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -839,13 +841,21 @@ cudaError_t launch_reduce_one(const DecodeParams& p, cudaStream_t st) {
     if (dev < 31) __atomic_fetch_or(&configured_devices, 1 << dev, __ATOMIC_ACQ_REL);
   }
   const dim3 grid(p.num_kv_heads * p.group, p.num_seqs);
-  return launch_pdl(kern, grid, dim3(kRedWarps * 32), smem, st, p);
+  return launch_pdl(kern, grid, dim3(W * 32), smem, st, p);
+}
+
+template <int D, bool kBf16>
+cudaError_t launch_reduce_d(const DecodeParams& p, cudaStream_t st) {
+  // Rows of at most one chunk: one warp, one stage (many rows per SM). Longer rows: two warps with
+  // four chunks in flight each.
+  if (p.ws_parts <= kRedChunk) return launch_reduce_one<D, kBf16, 1, 1>(p, st);
+  return launch_reduce_one<D, kBf16, 2, 4>(p, st);
 }
 
 cudaError_t launch_reduce(const DecodeConfig& c, const DecodeParams& p, cudaStream_t st) {
   const bool bf = c.q == QType::BF16;
-  if (c.head_dim == 128) return bf ? launch_reduce_one<128, true>(p, st) : launch_reduce_one<128, false>(p, st);
-  return bf ? launch_reduce_one<64, true>(p, st) : launch_reduce_one<64, false>(p, st);
+  if (c.head_dim == 128) return bf ? launch_reduce_d<128, true>(p, st) : launch_reduce_d<128, false>(p, st);
+  return bf ? launch_reduce_d<64, true>(p, st) : launch_reduce_d<64, false>(p, st);
 }
 
 uint32_t* decode_error_word() {
