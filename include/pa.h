@@ -264,7 +264,9 @@ size_t pa_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t 
  *     larger partition_tokens needs less.
  *   - The first call on a device that splits a context looks up the array's device address
  *     (cudaGetSymbolAddress, with that device current), after its argument checks, and caches it;
- *     make such a call before any stream capture.
+ *     make such a call before any stream capture. The cached address (like that of the library's
+ *     own error word) belongs to the device's context as it was then: a cudaDeviceReset of that
+ *     device after the first call is not supported in the same process.
  *   - The array takes PA_NO_ALLOC_SCRATCH_BYTES (32 MiB) on every device where the library's device
  *     code is loaded (depending on CUDA's module-loading mode, at start-up or at the latest on the
  *     first call), until the process exits.
