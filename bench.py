@@ -272,11 +272,15 @@ def measured_hbm_peak():
         return FALLBACK_HBM_GBS, "fallback (no MEASURED_PEAKS.json)"
 
 
+# The sources of the decode kernels whose DRAM traffic profiles/decode_traffic.json records.
+DECODE_SOURCES = ("decode.cu", "decode_math.cuh", "decode_units.cu", "pa_device.cuh", "internal.h")
+
+
 def decode_source_hash() -> str:
     """Hash of the decode kernel's sources with comments, blank lines and line-edge whitespace removed:
     the recorded DRAM traffic stays valid across comment edits and is dropped by any code change."""
     h = hashlib.sha256()
-    for f in ("decode.cu", "decode_math.cuh", "decode_units.cu", "pa_device.cuh", "internal.h"):
+    for f in DECODE_SOURCES:
         with open(os.path.join(ROOT, "paged_kv_cache_385_b200", "csrc", f), encoding="utf-8") as fh:
             text = re.sub(r"/\*.*?\*/", "", fh.read(), flags=re.S)
         lines = [re.sub(r"//.*$", "", ln).strip() for ln in text.splitlines()]

@@ -6,7 +6,7 @@ import shutil
 
 import bench
 
-SRC = ("decode.cu", "pa_device.cuh", "internal.h")
+SRC = bench.DECODE_SOURCES
 
 
 def _tree(tmp_path, edit=None):
