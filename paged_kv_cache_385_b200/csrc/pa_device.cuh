@@ -113,6 +113,29 @@ __device__ __forceinline__ uint64_t l2_evict_last_policy() {
   return pol;
 }
 
+// Named barrier `id` over `n` threads (a multiple of 32) that also returns whether `v` held in every
+// one of them. Every participating thread must reach it.
+__device__ __forceinline__ bool bar_and(int id, int n, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.and.pred p, %2, %3, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(v)), "r"(id), "r"(n)
+      : "memory");
+  return r != 0;
+}
+
+// 3-D tiled bulk tensor store shared -> global (bulk-group completion: commit, then wait_group).
+// x * elem_bytes must be a multiple of 16; no coordinate may be negative.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, uint32_t src, int32_t x, int32_t y, int32_t z) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4}], [%1];"
+               ::"l"(reinterpret_cast<uint64_t>(map)), "r"(src), "r"(x), "r"(y), "r"(z)
+               : "memory");
+}
+
 // tma_load_2d with an L2 cache policy.
 __device__ __forceinline__ void tma_load_2d_hint(uint32_t dst, const CUtensorMap* map, uint32_t bar, int32_t x, int32_t y,
                                                  uint64_t policy) {

@@ -78,7 +78,8 @@ __device__ __forceinline__ float extreme(const float (&v)[n]) {
 template <bool kBf16, bool kPrefix>
 __global__ void __launch_bounds__(kThreads, 2)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
-                      const __grid_constant__ CUtensorMap vmap, const MqParams p) {
+                      const __grid_constant__ CUtensorMap vmap, const __grid_constant__ CUtensorMap omap,
+                      const MqParams p) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t base = smem_u32(smem);
   if (base & 1023u) {  // the swizzled tiles need 1024-byte alignment; never seen, but do not guess
@@ -382,9 +383,14 @@ __global__ void __launch_bounds__(kThreads, 2)
       // return early while the previous P.V is still pending, since O_done may then be two phases back.)
       const bool done = __all_sync(kFull, mbar_wait_bounded(B(kAllDone), 0, deadline));
       if (done) tc05::fence_after_sync();
-      if (!done) {
-        ok = false;
-      } else if constexpr (kPrefix) {
+      if (!done) ok = false;
+    }
+    // A full prefill tile leaves as tensor stores once all four softmax warps agree: every one of
+    // them reaches this reducing barrier, so none waits at the staging barrier below for a warp that
+    // gave up.
+    const bool tma_out = !kPrefix && (tile + 1) * kRows <= num_rows && bar_and(1, 128, ok);
+    if (ok) {
+      if constexpr (kPrefix) {
         // O rows go through shared memory (the K/V stages are idle now) and leave it as one bulk
         // copy per 512-byte workspace row. (That every sequence maps the prefix pages to sequence 0's
         // blocks is checked by the suffix decode, off this kernel's critical path.)
@@ -413,6 +419,41 @@ __global__ void __launch_bounds__(kThreads, 2)
                        : "memory");
           asm volatile("cp.async.bulk.commit_group;" ::: "memory");
           asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");  // before the CTA's smem goes
+        }
+      } else if (tma_out) {
+        // A full tile leaves as two tensor stores (one per 64-column half) from the K stages, idle
+        // now: each row is written into the 128-byte-swizzled layout the output map names (16-byte
+        // chunk c of row r at position c ^ (r % 8)), so the rows go out coalesced, not as scattered
+        // 16-byte stores. A partial tile (its last rows would be the next sequence's) takes the
+        // per-row path below.
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        const uint32_t stg = base + kKOff;
+        static_assert(kKOff + kTile <= kVOff, "the output tile fits the K stages");
+#pragma unroll
+        for (int c = 0; c < kD / 32; ++c) {
+          float v[32];
+          tc05::ld32(tO + lane_off + c * 32, v);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int chunk = (c & 1) * 4 + q;  // 8 columns each, within the half c / 2
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(stg + (c >> 1) * kHalf + r * 128 +
+                                                                          ((chunk ^ (r & 7)) << 4)),
+                         "r"(pack2<kBf16>(v[8 * q] * inv, v[8 * q + 1] * inv)),
+                         "r"(pack2<kBf16>(v[8 * q + 2] * inv, v[8 * q + 3] * inv)),
+                         "r"(pack2<kBf16>(v[8 * q + 4] * inv, v[8 * q + 5] * inv)),
+                         "r"(pack2<kBf16>(v[8 * q + 6] * inv, v[8 * q + 7] * inv))
+                         : "memory");
+          }
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        asm volatile("bar.sync 1, 128;" ::: "memory");  // the four softmax warps' rows are staged
+        if (threadIdx.x == 0) {
+          const int tok0 = q_row0 + tile * (kRows / G);
+          tma_store_3d(&omap, stg, 0, hk * G, tok0);
+          tma_store_3d(&omap, stg + kHalf, 64, hk * G, tok0);
+          asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+          // Complete (not only read) before the CTA exits: the next grid may read out.
+          asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
         }
       } else {
         const float inv = l > 0.f ? 1.f / l : 0.f;
@@ -460,8 +501,8 @@ __global__ void __launch_bounds__(kThreads, 2)
 }
 
 template <bool kBf16, bool kPrefix>
-cudaError_t launch_tc(dim3 grid, const CUtensorMap& qm, const CUtensorMap& km, const CUtensorMap& vm, const MqParams& p,
-                      cudaStream_t st) {
+cudaError_t launch_tc(dim3 grid, const CUtensorMap& qm, const CUtensorMap& km, const CUtensorMap& vm,
+                      const CUtensorMap& om, const MqParams& p, cudaStream_t st) {
   auto kern = prefill_tc_kernel<kBf16, kPrefix>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
@@ -475,7 +516,7 @@ cudaError_t launch_tc(dim3 grid, const CUtensorMap& qm, const CUtensorMap& km, c
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, qm, km, vm, p);
+  return cudaLaunchKernelEx(&cfg, kern, qm, km, vm, om, p);
 }
 
 }  // namespace
@@ -485,12 +526,12 @@ bool prefill_tc_supported(int head_dim, int group) {
 }
 
 cudaError_t launch_prefill_tc(KvType kv, const CUtensorMap& qm, const CUtensorMap& km, const CUtensorMap& vm,
-                              const MqParams& p, int max_query_len, cudaStream_t st) {
+                              const CUtensorMap& om, const MqParams& p, int max_query_len, cudaStream_t st) {
   if (kv != KvType::F16 && kv != KvType::BF16) return cudaErrorInvalidValue;
   const int64_t rows = static_cast<int64_t>(max_query_len) * p.group;
   const dim3 grid(static_cast<unsigned>((rows + kRows - 1) / kRows), p.num_kv_heads, p.num_seqs);
-  return kv == KvType::BF16 ? launch_tc<true, false>(grid, qm, km, vm, p, st)
-                            : launch_tc<false, false>(grid, qm, km, vm, p, st);
+  return kv == KvType::BF16 ? launch_tc<true, false>(grid, qm, km, vm, om, p, st)
+                            : launch_tc<false, false>(grid, qm, km, vm, om, p, st);
 }
 
 // Shared-prefix mode: grid (row tiles of num_seqs * G, KV heads, prefix chunks); chunk_tokens must be
@@ -501,8 +542,9 @@ cudaError_t launch_prefix_tc(KvType kv, const CUtensorMap& qm, const CUtensorMap
   if (p.chunk_tokens <= 0 || p.chunk_tokens % kKeys || p.prefix_tokens % 16) return cudaErrorInvalidValue;
   const int64_t rows = static_cast<int64_t>(p.num_seqs) * p.group;
   const dim3 grid(static_cast<unsigned>((rows + kRows - 1) / kRows), p.num_kv_heads, p.num_chunks);
-  return kv == KvType::BF16 ? launch_tc<true, true>(grid, qm, km, vm, p, st)
-                            : launch_tc<false, true>(grid, qm, km, vm, p, st);
+  // (The output map is not used in this mode: partials leave through the workspace.)
+  return kv == KvType::BF16 ? launch_tc<true, true>(grid, qm, km, vm, qm, p, st)
+                            : launch_tc<false, true>(grid, qm, km, vm, qm, p, st);
 }
 
 }  // namespace pa
