@@ -124,6 +124,7 @@ struct MqParams {
   void* out;                   // prefill: [T, Hq, D]
   int64_t o_stride_t, o_stride_h;
   uint32_t* err;
+  int32_t row_tiles, num_items;  // tcgen05 kernels: 128-row tiles per sequence (or per prefix chunk), work items
 };
 constexpr int kPrefixChunkTokens = 256;
 cudaError_t launch_prefix(KvType kv, int head_dim, const CUtensorMap& k_map, const CUtensorMap& v_map,

@@ -150,6 +150,19 @@ __device__ __forceinline__ void st32u(uint32_t taddr, const uint32_t (&w)[32]) {
       : "memory");
 }
 
+// 16 consecutive 32-bit columns per lane from registers (raw words); no wait (tcgen05.wait::st, or
+// st_wait below, must follow before the data is relied on).
+__device__ __forceinline__ void st16u_nowait(uint32_t taddr, const uint32_t* w) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16};"
+      ::"r"(taddr), "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7]), "r"(w[8]),
+        "r"(w[9]), "r"(w[10]), "r"(w[11]), "r"(w[12]), "r"(w[13]), "r"(w[14]), "r"(w[15])
+      : "memory");
+}
+
+__device__ __forceinline__ void st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
 // 3-D tiled TMA load (box {x, y, z}), completion on an mbarrier; x * elem must be a multiple of 16.
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int32_t x, int32_t y,
                                             int32_t z) {
