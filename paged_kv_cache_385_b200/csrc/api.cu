@@ -147,6 +147,25 @@ int encode_q_map(CUtensorMap* map, const pa_tensor* q, int group) {
   return PA_OK;
 }
 
+// The split workspace's partial rows ws_acc [B, Hq, P, D] (float32) as a 4-D tensor {D, P, Hq, B},
+// boxes of 32 x 1 x G x (128 / G): 128 rows (sequences x group heads of one KV head, one partition) of
+// 32 columns, 128-byte swizzle. The workspace is 256-byte aligned and D * 4 is a multiple of 16.
+int encode_ws_map(CUtensorMap* map, float* ws_acc, int64_t B, int64_t Hq, int64_t P, int64_t D, int group) {
+  auto fn = encode_fn();
+  if (!fn) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(P), static_cast<cuuint64_t>(Hq),
+                              static_cast<cuuint64_t>(B)};
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(D * 4), static_cast<cuuint64_t>(P * D * 4),
+                                 static_cast<cuuint64_t>(Hq * P * D * 4)};
+  const cuuint32_t box[4] = {32, 1, static_cast<cuuint32_t>(group), static_cast<cuuint32_t>(128 / group)};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, ws_acc, dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled (workspace) failed (%d)", static_cast<int>(r));
+  return PA_OK;
+}
+
 // Host-side fault injection (pa_debug_fail_next_launches): calls left that fail as a launch would.
 std::atomic<int32_t> g_injected_failures{0};
 
@@ -594,9 +613,11 @@ static int decode_impl(pa_tensor* out, const pa_tensor* q, const pa_tensor* k_ca
     pp.ws_parts = p.ws_parts;
     pp.err = p.err;
     if (use_tc_prefix) {
-      CUtensorMap qm;
-      if ((st = encode_q_map(&qm, q, static_cast<int>(G)))) return st;
-      e = pa::launch_prefix_tc(cfg.kv, qm, km, vm, pp, s);
+      CUtensorMap qm, wm;
+      if ((st = encode_q_map(&qm, q, static_cast<int>(G))) ||
+          (st = encode_ws_map(&wm, pp.ws_acc, B, Hq, ws_parts, D, static_cast<int>(G))))
+        return st;
+      e = pa::launch_prefix_tc(cfg.kv, qm, km, vm, wm, pp, s);
     } else {
       e = pa::launch_prefix(cfg.kv, cfg.head_dim, km, vm, pp, s);
     }

@@ -113,6 +113,14 @@ __device__ __forceinline__ uint64_t l2_evict_last_policy() {
   return pol;
 }
 
+// 4-D tiled bulk tensor store shared -> global (bulk-group completion); same rules as tma_store_3d.
+__device__ __forceinline__ void tma_store_4d(const CUtensorMap* map, uint32_t src, int32_t x, int32_t y, int32_t z,
+                                             int32_t w) {
+  asm volatile("cp.async.bulk.tensor.4d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4, %5}], [%1];"
+               ::"l"(reinterpret_cast<uint64_t>(map)), "r"(src), "r"(x), "r"(y), "r"(z), "r"(w)
+               : "memory");
+}
+
 // Named barrier `id` over `n` threads (a multiple of 32) that also returns whether `v` held in every
 // one of them. Every participating thread must reach it.
 __device__ __forceinline__ bool bar_and(int id, int n, bool v) {

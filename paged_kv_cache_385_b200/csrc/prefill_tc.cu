@@ -218,13 +218,13 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (lane == 0) {
       prefetch_tensormap(&qmap);
       int g = 0, it = 0;
-      for (int k = 0; ok; ++k) {
-        const uint64_t deadline = globaltimer_ns() + 2000000000ull;
+      for (int k = 0; ok && (!kPrefix || k == 0); ++k) {  // (a prefix CTA takes one item)
         const int64_t w64 = static_cast<int64_t>(k) * gridDim.x + blockIdx.x;
         if (w64 >= p.num_items) break;
         const int w = static_cast<int>(w64);
         const Item I = item(w);
         if (I.nkb == 0) continue;
+        const uint64_t deadline = globaltimer_ns() + 2000000000ull;
         // Q(it) once every QK of the previous item has run (the issuer commits Q_empty after them).
         if (it > 0 && !mbar_wait_bounded(B(kQEmpty), (it - 1) & 1, deadline)) {
           ok = false;
@@ -252,7 +252,15 @@ __global__ void __launch_bounds__(kThreads, 2)
       // read out: wait for the softmax warps' Staged arrival, issue its stores, and wait for their reads.
       auto drain_staged = [&](const Item& I, int i, uint64_t deadline) -> bool {
         if (!mbar_wait_bounded(B(kStaged), i & 1, deadline)) return false;
-        if (full_tile(I)) {
+        if constexpr (kPrefix) {
+          // The partial tile, from the K/V stages: boxes of 32 columns x this chunk's partition x G
+          // heads x 128 / G sequences (those past the batch are clipped by the map).
+#pragma unroll
+          for (int c = 0; c < kD / 32; ++c)
+            tma_store_4d(&omap, base + kKOff + c * (kRows * 128), 32 * c, I.s, I.hk * G, I.tile * (kRows / G));
+          asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+          asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+        } else if (full_tile(I)) {
           const int tok0 = I.q_row0 + I.tile * (kRows / G);
           tma_store_3d(&omap, base + kVOff, 0, I.hk * G, tok0);
           tma_store_3d(&omap, base + kVOff + kHalf, 64, I.hk * G, tok0);
@@ -263,13 +271,13 @@ __global__ void __launch_bounds__(kThreads, 2)
       };
       int g = 0, it = 0;
       Item prev{};
-      for (int k = 0; ok; ++k) {
-        const uint64_t deadline = globaltimer_ns() + 2000000000ull;
+      for (int k = 0; ok && (!kPrefix || k == 0); ++k) {  // (a prefix CTA takes one item)
         const int64_t w64 = static_cast<int64_t>(k) * gridDim.x + blockIdx.x;
         if (w64 >= p.num_items) break;
         const int w = static_cast<int>(w64);
         const Item I = item(w);
         if (I.nkb == 0) continue;
+        const uint64_t deadline = globaltimer_ns() + 2000000000ull;
         if (it > 0 && !drain_staged(prev, it - 1, deadline)) {
           ok = false;
           break;
@@ -283,8 +291,8 @@ __global__ void __launch_bounds__(kThreads, 2)
         prev = I;
       }
       if (ok && it > 0) ok = drain_staged(prev, it - 1, globaltimer_ns() + 2000000000ull);
-      // Complete (not only read) before the CTA exits: the next grid may read out.
-      asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+      // (Every store has read its shared-memory source by here; the global writes are the grid's
+      // own memory operations, visible to a stream-ordered or dependent grid once this one completes.)
       if (!ok) atomicOr(p.err, 4u);
     }
   } else if (warp == 5) {
@@ -292,13 +300,13 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (lane == 0) {
       constexpr uint32_t idesc_qk = tc05::idesc_f16(kBf16, kRows, kKeys, false, false);
       int g = 0, it = 0;
-      for (int k = 0; ok; ++k) {
-        const uint64_t deadline = globaltimer_ns() + 2000000000ull;
+      for (int k = 0; ok && (!kPrefix || k == 0); ++k) {  // (a prefix CTA takes one item)
         const int64_t w64 = static_cast<int64_t>(k) * gridDim.x + blockIdx.x;
         if (w64 >= p.num_items) break;
         const int w = static_cast<int>(w64);
         const Item I = item(w);
         if (I.nkb == 0) continue;
+        const uint64_t deadline = globaltimer_ns() + 2000000000ull;
         // Q_full next completes for Q(it+1), loaded only after this item's QKs: the wait is exact.
         ok = mbar_wait_bounded(B(kQFull), it & 1, deadline);
         for (int j = 0; j < I.nkb && ok; ++j) {
@@ -338,13 +346,13 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (lane == 0) {
       constexpr uint32_t idesc_pv = tc05::idesc_f16(kBf16, kRows, kD, false, true);
       int g = 0, it = 0;
-      for (int k = 0; ok; ++k) {
-        const uint64_t deadline = globaltimer_ns() + 2000000000ull;
+      for (int k = 0; ok && (!kPrefix || k == 0); ++k) {  // (a prefix CTA takes one item)
         const int64_t w64 = static_cast<int64_t>(k) * gridDim.x + blockIdx.x;
         if (w64 >= p.num_items) break;
         const int w = static_cast<int>(w64);
         const Item I = item(w);
         if (I.nkb == 0) continue;
+        const uint64_t deadline = globaltimer_ns() + 2000000000ull;
         // The item's first P.V overwrites O: the previous item's epilogue must have read it. O_free next
         // completes for this item's epilogue, which needs these products: the wait is exact.
         if (it > 0 && !mbar_wait_bounded(B(kOFree), (it - 1) & 1, deadline)) ok = false;
@@ -383,13 +391,13 @@ __global__ void __launch_bounds__(kThreads, 2)
     const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
     const float sl2 = p.score_scale_log2;
     int g = 0;
-    for (int k = 0; ok; ++k) {
-      const uint64_t deadline = globaltimer_ns() + 2000000000ull;
+    for (int k = 0; ok && (!kPrefix || k == 0); ++k) {  // (a prefix CTA takes one item)
       const int64_t w64 = static_cast<int64_t>(k) * gridDim.x + blockIdx.x;
       if (w64 >= p.num_items) break;
       const int w = static_cast<int>(w64);
       const Item I = item(w);
       if (I.nkb == 0) continue;
+      const uint64_t deadline = globaltimer_ns() + 2000000000ull;
       const int R = I.tile * kRows + r;
       const bool valid = R < I.num_rows;
       // The row's visible keys, counted from key0: the causal diagonal, or the sequence's context
@@ -510,35 +518,30 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
       tc05::fence_after_sync();
       if constexpr (kPrefix) {
-        // The row's (m, l, O) -> its workspace slot. O rows go through shared memory (the K/V stages:
-        // a prefix CTA takes one item, so nothing is prefetched into them) and leave it as one bulk
-        // copy per 512-byte workspace row. (That every sequence maps the prefix pages to sequence 0's
-        // blocks is checked by the suffix decode, off this kernel's critical path.)
-        constexpr uint32_t kRowStride = (kD + 4) * 4;  // padded: row-wise writes free of bank conflicts
-        const uint32_t stg = base + kKOff + warp * 32 * kRowStride;
-        static_assert(kKOff + 4 * 32 * kRowStride <= kBarOff, "staging fits the K/V stages");
+        // The row's (m, l, O) -> its workspace slot. O goes through shared memory (the K/V stages: a
+        // prefix CTA takes one item, so nothing is prefetched into them) as four 32-column boxes in
+        // the 128-byte-swizzled layout the workspace map names (16-byte chunk c of row r at position
+        // c ^ (r % 8), conflict-free), which the V producer lane stores as tensor stores; (m, l)
+        // directly. (That every sequence maps the prefix pages to sequence 0's blocks is checked by
+        // the suffix decode, off this kernel's critical path.)
+        const uint32_t stg = base + kKOff;
+        static_assert(kKOff + (kD / 32) * kRows * 128 <= kBarOff, "the partial tile fits the K/V stages");
 #pragma unroll
         for (int c = 0; c < kD / 32; ++c) {
           float v[32];
           tc05::ld32(tO + lane_off + c * 32, v);
 #pragma unroll
           for (int q = 0; q < 8; ++q)
-            asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(stg + lane * kRowStride + (c * 32 + 4 * q) * 4),
+            asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(stg + c * (kRows * 128) + r * 128 +
+                                                                           ((q ^ (r & 7)) << 4)),
                          "f"(v[4 * q]), "f"(v[4 * q + 1]), "f"(v[4 * q + 2]), "f"(v[4 * q + 3])
                          : "memory");
         }
-        // Each valid row's lane issues the bulk copy of its own staged row (512 bytes, 16-byte
-        // aligned at both ends), after a proxy fence makes its shared-memory writes visible to it.
-        const int Hq = p.num_kv_heads * G;
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         if (valid) {
+          const int Hq = p.num_kv_heads * G;
           const int64_t slot = (static_cast<int64_t>(R / G) * Hq + I.hk * G + R % G) * p.ws_parts + I.s;
           *reinterpret_cast<float2*>(p.ws_ml + slot * 2) = make_float2(m, l);
-          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-          asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(p.ws_acc + slot * kD),
-                       "r"(stg + lane * kRowStride), "r"(kD * 4)
-                       : "memory");
-          asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-          asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");  // before the CTA's smem goes
         }
       } else {
         const float inv = l > 0.f ? 1.f / l : 0.f;
@@ -677,10 +680,10 @@ cudaError_t launch_prefill_tc(KvType kv, const CUtensorMap& qm, const CUtensorMa
                             : launch_tc<false, false>(grid, qm, km, vm, om, q, st);
 }
 
-// Shared-prefix mode: grid (row tiles of num_seqs * G, KV heads, prefix chunks); chunk_tokens must be
-// a multiple of the key block.
+// Shared-prefix mode: one CTA per (row tile of num_seqs * G, KV head, prefix chunk); chunk_tokens must
+// be a multiple of the key block. wm maps the workspace's partial rows.
 cudaError_t launch_prefix_tc(KvType kv, const CUtensorMap& qm, const CUtensorMap& km, const CUtensorMap& vm,
-                             const MqParams& p, cudaStream_t st) {
+                             const CUtensorMap& wm, const MqParams& p, cudaStream_t st) {
   if (kv != KvType::F16 && kv != KvType::BF16) return cudaErrorInvalidValue;
   if (p.chunk_tokens <= 0 || p.chunk_tokens % kKeys || p.prefix_tokens % 16) return cudaErrorInvalidValue;
   // One item per CTA: (row tile of num_seqs * G, KV head, prefix chunk).
@@ -690,9 +693,8 @@ cudaError_t launch_prefix_tc(KvType kv, const CUtensorMap& qm, const CUtensorMap
   MqParams q = p;
   q.row_tiles = static_cast<int32_t>(tiles);
   q.num_items = static_cast<int32_t>(items);
-  // (The output map is not used in this mode: partials leave through the workspace.)
-  return kv == KvType::BF16 ? launch_tc<true, true>(static_cast<int>(items), qm, km, vm, qm, q, st)
-                            : launch_tc<false, true>(static_cast<int>(items), qm, km, vm, qm, q, st);
+  return kv == KvType::BF16 ? launch_tc<true, true>(static_cast<int>(items), qm, km, vm, wm, q, st)
+                            : launch_tc<false, true>(static_cast<int>(items), qm, km, vm, wm, q, st);
 }
 
 }  // namespace pa
