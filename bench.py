@@ -635,8 +635,7 @@ def run_prefill(args, rank, world, local_rank):
                        "flops_per_call": flops},
             "roofline": {"bound": "tensor", "achieved": round(tflops, 1), "peak": peak, "unit": "TFLOP/s",
                          "frac": round(tflops / peak, 4), "traffic": None, "peak_source": src,
-                         "kernel": {0: "warp-level mma.sync", 1: "tcgen05 (tensor memory accumulators)",
-                                    2: "tcgen05, two tiles per CTA alternating softmax and MMAs"}[kernel]},
+                         "kernel": "tcgen05 (tensor memory accumulators)" if kernel == 1 else "warp-level mma.sync"},
             "gpu_launches": K, "clocks": clocks.summary()}), flush=True)
 
 

@@ -223,9 +223,7 @@ size_t pa_decode_cascade_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, 
  *                 sequence s including the chunk (n_s <= context_lens[s] <= 16 * max_blocks).
  *   max_query_len host-known bound on n_s (sizes the grid without a device read).
  *   kernel        -1 = choose (tcgen05 when D = 128 and Hq / Hkv <= 16 divides 128), 0 = warp-level mma.sync
- *                 tiles, 1 = tcgen05 (5th-generation tensor cores, accumulators in tensor memory),
- *                 2 = tcgen05 with two 128-row tiles per CTA whose softmax and MMAs alternate (same
- *                 support condition as 1; PA_ERR_UNSUPPORTED where it does not hold).
+ *                 tiles, 1 = tcgen05 (5th-generation tensor cores, accumulators in tensor memory).
  * Row i of sequence s is position p = context_lens[s] - n_s + i and sees positions 0 .. p:
  * out = softmax(scale * q K[0..p]^T) V[0..p], float32 accumulation, rounded to nearest even.
  * Violations only the device can see (n_s > context_lens[s], n_s > max_query_len) set

@@ -24,8 +24,8 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libpagedattn.so")
 
-SOURCES = ["api.cu", "decode.cu", "decode_units.cu", "multiquery.cu", "prefill_tc.cu", "prefill_pp.cu", "cache.cu",
-           "no_alloc.cu", "selftest.cu", "allocator.cpp"]
+SOURCES = ["api.cu", "decode.cu", "decode_units.cu", "multiquery.cu", "prefill_tc.cu", "cache.cu", "no_alloc.cu",
+           "selftest.cu", "allocator.cpp"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2", "-I" + INCLUDE, "-I" + CSRC,
               "--expt-relaxed-constexpr", "-Xptxas", "-warn-spills"]

@@ -1,7 +1,6 @@
 // C-ABI entry points of libpagedattn: argument validation, TMA descriptor encoding, dispatch.
 // Host code only. Every argument error is found here before the first device call; the kernels
-// live in decode.cu, decode_units.cu, multiquery.cu, prefill_tc.cu, prefill_pp.cu, cache.cu, no_alloc.cu and
-// selftest.cu.
+// live in decode.cu, decode_units.cu, multiquery.cu, prefill_tc.cu, cache.cu, no_alloc.cu and selftest.cu.
 #include <cudaTypedefs.h>
 
 #include <atomic>
@@ -766,9 +765,9 @@ int pa_prefill(pa_tensor* out, const pa_tensor* q, const pa_tensor* k_cache, con
     return fail(PA_ERR_INVALID_ARG, "NULL data pointer");
   // The kernel choice is an argument error, reported before any device call.
   const int G = static_cast<int>(Hq / num_kv_heads);
-  if (kernel < -1 || kernel > 2) return fail(PA_ERR_INVALID_ARG, "kernel must be -1, 0, 1 or 2");
+  if (kernel < -1 || kernel > 1) return fail(PA_ERR_INVALID_ARG, "kernel must be -1, 0 or 1");
   const bool tc_ok = pa::prefill_tc_supported(static_cast<int>(D), G);
-  if (kernel >= 1 && !tc_ok) return fail(PA_ERR_UNSUPPORTED, "the tcgen05 prefill needs head_dim 128 and a group of at most 16 dividing 128");
+  if (kernel == 1 && !tc_ok) return fail(PA_ERR_UNSUPPORTED, "the tcgen05 prefill needs head_dim 128 and a group of at most 16 dividing 128");
   pa::MqParams p{};
   p.q = q->data;
   p.q_stride_s = q->stride[0];
@@ -793,11 +792,10 @@ int pa_prefill(pa_tensor* out, const pa_tensor* q, const pa_tensor* k_cache, con
   if ((st = encode_pool_map(&km, k_cache, 2)) || (st = encode_pool_map(&vm, v_cache, 2))) return st;
   const pa::KvType kv = cd == PA_BF16 ? pa::KvType::BF16 : pa::KvType::F16;
   cudaError_t e;
-  if (kernel >= 1 || (kernel == -1 && tc_ok)) {
+  if (kernel == 1 || (kernel == -1 && tc_ok)) {
     CUtensorMap qm, om;
     if ((st = encode_q_map(&qm, q, G)) || (st = encode_q_map(&om, out, G))) return st;
-    e = kernel == 2 ? pa::launch_prefill_pp(kv, qm, km, vm, p, max_query_len, static_cast<cudaStream_t>(stream))
-                    : pa::launch_prefill_tc(kv, qm, km, vm, om, p, max_query_len, static_cast<cudaStream_t>(stream));
+    e = pa::launch_prefill_tc(kv, qm, km, vm, om, p, max_query_len, static_cast<cudaStream_t>(stream));
   } else {
     e = pa::launch_prefill(kv, static_cast<int>(D), km, vm, p, max_query_len, static_cast<cudaStream_t>(stream));
   }

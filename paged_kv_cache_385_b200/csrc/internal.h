@@ -136,10 +136,6 @@ cudaError_t launch_prefill(KvType kv, int head_dim, const CUtensorMap& k_map, co
 bool prefill_tc_supported(int head_dim, int group);
 cudaError_t launch_prefill_tc(KvType kv, const CUtensorMap& q_map, const CUtensorMap& k_map, const CUtensorMap& v_map,
                               const CUtensorMap& o_map, const MqParams& p, int max_query_len, cudaStream_t stream);
-// Two-tile tcgen05 prefill (prefill_pp.cu): one CTA per SM holding two 128-row tiles whose softmax
-// and MMAs alternate; same maps and support condition as launch_prefill_tc.
-cudaError_t launch_prefill_pp(KvType kv, const CUtensorMap& q_map, const CUtensorMap& k_map, const CUtensorMap& v_map,
-                              const MqParams& p, int max_query_len, cudaStream_t stream);
 // The same kernel in shared-prefix mode: q_map over q [B, Hq, D], partials to ws slots 0 .. num_chunks-1;
 // ws_map is a 4-D map over ws_acc {D, P, Hq, B} (float32) with box {32, 1, G, 128 / G}, 128-byte swizzle.
 cudaError_t launch_prefix_tc(KvType kv, const CUtensorMap& q_map, const CUtensorMap& k_map, const CUtensorMap& v_map,

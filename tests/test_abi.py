@@ -177,7 +177,7 @@ def test_cascade_option_validation_happens_on_the_host():
 
 
 def test_prefill_kernel_choice_is_checked_on_the_host():
-    """The tcgen05 prefills take head_dim 128 and a group dividing 128: asking for either with D = 64 is
+    """The tcgen05 prefill takes head_dim 128 and a group dividing 128: asking for it with D = 64 is
     refused before any device work; an unknown kernel number too."""
     T, Hq, Hkv, D, NB, B = 8, 4, 4, 64, 4, 1
     q = aligned_zeros((T, Hq, D), torch.float16)
@@ -189,10 +189,9 @@ def test_prefill_kernel_choice_is_checked_on_the_host():
                                                             (qs, "qs"), (lens, "lens"))]
     lib = pa.lib()
     args = [ctypes.byref(t) for t in ts]
-    for kernel in (1, 2):  # both tcgen05 forms
-        assert lib.pa_prefill(*args, T, 0.125, Hkv, kernel, None) == pa.PA_ERR_UNSUPPORTED
-        assert "tcgen05" in pa.pa_last_error()
-    for kernel in (3, -2):
+    assert lib.pa_prefill(*args, T, 0.125, Hkv, 1, None) == pa.PA_ERR_UNSUPPORTED
+    assert "tcgen05" in pa.pa_last_error()
+    for kernel in (2, -2):
         assert lib.pa_prefill(*args, T, 0.125, Hkv, kernel, None) == pa.PA_ERR_INVALID_ARG
 
 

@@ -66,11 +66,11 @@ CASES = [
 ]
 
 
-@pytest.mark.parametrize("kernel", [0, 1, 2])
+@pytest.mark.parametrize("kernel", [0, 1])
 @pytest.mark.parametrize("ctxs,news,hq,hkv,d,dtype", CASES)
 def test_prefill_matches_oracle(ctxs, news, hq, hkv, d, dtype, kernel):
-    if kernel >= 1 and d != 128:
-        pytest.skip("the tcgen05 prefills take head_dim 128")
+    if kernel == 1 and d != 128:
+        pytest.skip("the tcgen05 prefill takes head_dim 128")
     bt, kc, vc, q, qs, host = _build(ctxs, news, hq, hkv, d, dtype, seed=sum(ctxs))
     out = torch.full((q.shape[0], hq, d), float("nan"), dtype=dtype, device="cuda")
     pa.pa_prefill(out, q.cuda(), kc, vc, bt.cuda(), qs.cuda(), torch.tensor(ctxs, dtype=torch.int32).cuda(),
@@ -86,7 +86,7 @@ def test_prefill_matches_oracle(ctxs, news, hq, hkv, d, dtype, kernel):
     assert np.array_equal(vc.view(torch.uint8).reshape(vp.shape).cpu().numpy(), vp)
 
 
-@pytest.mark.parametrize("kernel", [0, 1, 2])
+@pytest.mark.parametrize("kernel", [0, 1])
 @pytest.mark.parametrize("scale", [-0.11, 0.0, 1.5])
 def test_prefill_scale_sign_and_size(scale, kernel):
     """Negative and zero scales (the softmax max comes from the raw min, or every weight is equal) and
@@ -107,7 +107,7 @@ def test_tcgen05_and_warp_mma_prefill_agree():
     ctxs, news, hq, hkv, d = [1000, 77], [1000, 77], 32, 8, 128
     bt, kc, vc, q, qs, _ = _build(ctxs, news, hq, hkv, d, torch.bfloat16, seed=31)
     outs = []
-    for kernel in (0, 1, 2):
+    for kernel in (0, 1):
         out = torch.empty(q.shape[0], hq, d, dtype=torch.bfloat16, device="cuda")
         pa.pa_prefill(out, q.cuda(), kc, vc, bt.cuda(), qs.cuda(), torch.tensor(ctxs, dtype=torch.int32).cuda(),
                       max(news), d ** -0.5, hkv, kernel=kernel)
@@ -120,8 +120,7 @@ def test_tcgen05_and_warp_mma_prefill_agree():
         assert (outs[0].double() - o.double()).abs().max().item() <= 2 * TOL["bf16"]
 
 
-@pytest.mark.parametrize("kernel", [1, 2])
-def test_tcgen05_prefill_is_deterministic(kernel):
+def test_tcgen05_prefill_is_deterministic():
     """Repeated launches give bit-identical outputs: a pipeline race (a buffer reused before the MMA
     reading it finished) shows up as run-to-run differences, even where it stays within tolerance."""
     ctxs, news, hq, hkv, d = [2000, 1500, 333], [2000, 700, 333], 32, 8, 128
@@ -130,7 +129,7 @@ def test_tcgen05_prefill_is_deterministic(kernel):
     outs = []
     for _ in range(6):
         out = torch.empty(q.shape[0], hq, d, dtype=torch.bfloat16, device="cuda")
-        pa.pa_prefill(out, q.cuda(), kc, vc, bt.cuda(), qs.cuda(), lens, max(news), d ** -0.5, hkv, kernel=kernel)
+        pa.pa_prefill(out, q.cuda(), kc, vc, bt.cuda(), qs.cuda(), lens, max(news), d ** -0.5, hkv, kernel=1)
         outs.append(out)
     torch.cuda.synchronize()
     assert pa.pa_read_device_error(clear=True) == 0
@@ -168,7 +167,7 @@ def test_prefill_reports_impossible_chunks():
     assert pa.pa_read_device_error(clear=True) & pa.PA_DEVERR_CTX_RANGE
 
 
-@pytest.mark.parametrize("kernel", [0, 1, 2])
+@pytest.mark.parametrize("kernel", [0, 1])
 def test_permuted_physical_blocks_give_bit_identical_prefill(kernel):
     """The same logical K/V, q and chunks placed in two different sets of physical blocks."""
     ctxs, news, hq, hkv, d = [700, 5, 260, 1300], [400, 5, 131, 64], 32, 8, 128
