@@ -601,7 +601,7 @@ def run_prefill(args, rank, world, local_rank):
     btd = bt.to(device)
     # Causal FLOPs: QK^T and PV, 2 flops per MAC, position i sees i + 1 keys.
     flops = B * Hq * 2 * 2 * D * (n * (n + 1) // 2)
-    K, Wm = max(5, args.steps // 100), max(3, args.warmup)
+    K, Wm = max(20, args.steps // 100), max(3, args.warmup)
 
     kernel = 1 if args.kernel == -1 else args.kernel  # -1: the library's choice (tcgen05 here)
 
