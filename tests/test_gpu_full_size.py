@@ -110,3 +110,46 @@ def test_full_size_prefix_workload_every_output_and_pool_byte():
     k, v = dev.pool_bytes()
     assert np.array_equal(k, k_pool), f"K pool differs at {np.argwhere(k != k_pool)[:4]}"
     assert np.array_equal(v, v_pool), f"V pool differs at {np.argwhere(v != v_pool)[:4]}"
+
+
+def test_full_size_prefill_sampled_rows():
+    """The prefill the bench times (8 sequences x 2048-token prompts, Llama-3-8B heads 32/8, D=128,
+    bf16, the library's kernel choice: the persistent tcgen05 kernel with 16 items per CTA) against the
+    oracle's row definition on sampled rows: the first and last tokens of every sequence, tokens on
+    either side of a 128-row tile edge and inside the causal diagonal block, for query heads at both
+    ends of a KV group. The oracle reads the host K/V draws; every output is checked finite."""
+    B, n, Hq, Hkv, D = 8, 2048, 32, 8, 128
+    g = torch.Generator().manual_seed(4242)
+    nb = B * n // 16 + 9
+    order = torch.randperm(nb, generator=g)
+    alloc = pa.BlockAllocator(nb, order.tolist())
+    bt = pa.build_block_tables(alloc, [n] * B, n // 16)
+    assert np.array_equal(bt.numpy(), paging.build_block_tables([n] * B, order.numpy(), nb, 16, 0, n // 16))
+    K = torch.randn(B * n, Hkv, D, generator=g).to(torch.bfloat16)
+    V = torch.randn(B * n, Hkv, D, generator=g).to(torch.bfloat16)
+    q = torch.randn(B * n, Hq, D, generator=g).to(torch.bfloat16)
+    kc = torch.randint(0, 256, (nb, Hkv, 16, 2 * D), generator=g, dtype=torch.uint8).view(torch.bfloat16)
+    kc = kc.view(nb, Hkv, 16, D).cuda()
+    vc = torch.randint(0, 256, (nb, Hkv, 16, 2 * D), generator=g, dtype=torch.uint8).view(torch.bfloat16)
+    vc = vc.view(nb, Hkv, 16, D).cuda()
+    seqs = [s for s in range(B) for _ in range(n)]
+    poss = [t for _ in range(B) for t in range(n)]
+    pa.pa_reshape_and_cache(K.cuda(), V.cuda(), pa.pa_slots_for_positions(bt, seqs, poss).cuda(), kc, vc)
+    out = torch.full((B * n, Hq, D), float("nan"), dtype=torch.bfloat16, device="cuda")
+    qs = torch.arange(0, B * n + 1, n, dtype=torch.int32).cuda()
+    lens = torch.full((B,), n, dtype=torch.int32).cuda()
+    pa.pa_prefill(out, q.cuda(), kc, vc, bt.cuda(), qs, lens, n, D ** -0.5, Hkv)
+    torch.cuda.synchronize()
+    assert pa.pa_read_device_error(clear=True) == 0
+    got = out.float().cpu()
+    assert torch.isfinite(got).all()
+    worst = 0.0
+    for s in range(B):
+        Kd = oracle_case.values64(K[s * n:(s + 1) * n])
+        Vd = oracle_case.values64(V[s * n:(s + 1) * n])
+        for t in (0, 1, 31, 32, 1023, 1024, 2015, 2047):  # 32 tokens x 4 heads = one 128-row tile
+            qd = oracle_case.values64(q[s * n + t])
+            for h in (0, 3, 4, 31):
+                want = attention.decode_logical_one(qd[h], Kd[:t + 1], Vd[:t + 1], h, Hq, Hkv, D ** -0.5)
+                worst = max(worst, float(np.max(np.abs(got[s * n + t, h].double().numpy() - want))))
+    assert worst <= TOL["bf16"], worst

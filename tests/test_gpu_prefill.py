@@ -63,6 +63,9 @@ CASES = [
     ([129, 40], [129, 40], 4, 4, 128, torch.float16),
     # Long enough (24 key blocks) that the S / P buffers of the tcgen05 kernel are reused many times.
     ([1500, 300], [1500, 100], 8, 2, 128, torch.bfloat16),
+    # 696 row tiles x KV heads: more items than the persistent grid's 2 x SMs CTAs, so each CTA walks
+    # two or three items and hands Q, O and its rings from one to the next.
+    ([900, 1200, 640], [900, 600, 640], 32, 8, 128, torch.bfloat16),
 ]
 
 
