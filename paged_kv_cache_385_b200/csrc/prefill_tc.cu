@@ -134,7 +134,8 @@ __global__ void __launch_bounds__(kThreads, 2)
   // Work item w: (row tile, KV head, z). Prefill: z is the sequence, and items are numbered longest
   // first (the last row tiles of every sequence before the earlier ones); CTA c takes items c,
   // c + gridDim.x, ..., so every CTA starts on long items and ends on short ones. Prefix: z is the
-  // prefix chunk and row R of the grid is (sequence R / G, group head R % G); one item per CTA.
+  // prefix chunk and row R of the grid is (sequence R / G, group head R % G); one item per CTA, taken
+  // from the CTA's 3-D index.
   struct Item {
     int tile, hk, s;
     int q_row0, num_rows, start, key0, max_lim, npages, nkb;
@@ -144,9 +145,9 @@ __global__ void __launch_bounds__(kThreads, 2)
     Item I{};
     const int X = p.row_tiles;
     if constexpr (kPrefix) {
-      I.tile = w % X;
-      I.hk = (w / X) % p.num_kv_heads;
-      I.s = w / X / p.num_kv_heads;
+      I.tile = blockIdx.x;  // a 3-D grid of one item per CTA: (row tile, KV head, prefix chunk)
+      I.hk = blockIdx.y;
+      I.s = blockIdx.z;
       I.num_rows = p.num_seqs * G;
       if (I.tile * kRows >= I.num_rows) return I;
       I.key0 = I.s * p.chunk_tokens;
@@ -622,13 +623,13 @@ __global__ void __launch_bounds__(kThreads, 2)
 }
 
 template <bool kBf16, bool kPrefix>
-cudaError_t launch_tc(int grid, const CUtensorMap& qm, const CUtensorMap& km, const CUtensorMap& vm,
+cudaError_t launch_tc(dim3 grid, const CUtensorMap& qm, const CUtensorMap& km, const CUtensorMap& vm,
                       const CUtensorMap& om, const MqParams& p, cudaStream_t st) {
   auto kern = prefill_tc_kernel<kBf16, kPrefix>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.gridDim = grid;
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = kSmemBytes;
   cfg.stream = st;
@@ -675,7 +676,7 @@ cudaError_t launch_prefill_tc(KvType kv, const CUtensorMap& qm, const CUtensorMa
   MqParams q = p;
   q.row_tiles = static_cast<int32_t>(tiles);
   q.num_items = static_cast<int32_t>(items);
-  const int grid = static_cast<int>(std::min<int64_t>(items, 2 * static_cast<int64_t>(sms)));
+  const dim3 grid(static_cast<unsigned>(std::min<int64_t>(items, 2 * static_cast<int64_t>(sms))));
   return kv == KvType::BF16 ? launch_tc<true, false>(grid, qm, km, vm, om, q, st)
                             : launch_tc<false, false>(grid, qm, km, vm, om, q, st);
 }
@@ -689,12 +690,13 @@ cudaError_t launch_prefix_tc(KvType kv, const CUtensorMap& qm, const CUtensorMap
   // One item per CTA: (row tile of num_seqs * G, KV head, prefix chunk).
   const int64_t tiles = (static_cast<int64_t>(p.num_seqs) * p.group + kRows - 1) / kRows;
   const int64_t items = tiles * p.num_kv_heads * p.num_chunks;
-  if (items > 0x7fffffff) return cudaErrorInvalidValue;
+  if (items > 0x7fffffff || p.num_kv_heads > 65535 || p.num_chunks > 65535) return cudaErrorInvalidValue;
   MqParams q = p;
   q.row_tiles = static_cast<int32_t>(tiles);
   q.num_items = static_cast<int32_t>(items);
-  return kv == KvType::BF16 ? launch_tc<true, true>(static_cast<int>(items), qm, km, vm, wm, q, st)
-                            : launch_tc<false, true>(static_cast<int>(items), qm, km, vm, wm, q, st);
+  const dim3 grid(static_cast<unsigned>(tiles), p.num_kv_heads, p.num_chunks);
+  return kv == KvType::BF16 ? launch_tc<true, true>(grid, qm, km, vm, wm, q, st)
+                            : launch_tc<false, true>(grid, qm, km, vm, wm, q, st);
 }
 
 }  // namespace pa
