@@ -66,6 +66,9 @@ CASES = [
     # 696 row tiles x KV heads: more items than the persistent grid's 2 x SMs CTAs, so each CTA walks
     # two or three items and hands Q, O and its rings from one to the next.
     ([900, 1200, 640], [900, 600, 640], 32, 8, 128, torch.bfloat16),
+    # Groups of 16 query heads (the largest the tcgen05 kernel takes: 8 tokens x 16 heads per tile),
+    # chunks that end mid-tile, one sequence with a single new token.
+    ([333, 70, 1], [101, 70, 1], 32, 2, 128, torch.float16),
 ]
 
 
