@@ -113,17 +113,11 @@ struct TcMath {
     }
   }
 
-  // One 16-token page; kb/vb are the shared addresses of its K and V pages; nv valid tokens.
-  __device__ __forceinline__ void page(uint32_t kb, uint32_t vb, int nv, float sl2) {
+  // S^T = K . Q^T of one 16-token page (K page at shared address kb) into sc.
+  __device__ __forceinline__ void qk(uint32_t kb, float (&sc)[NT][4]) {
     const int x7 = lane & 7;
     const int a_tok = tok_of_row((((lane >> 3) & 1) << 3) | x7);  // K matrices: row half = bit 3
     const int a_co = lane >> 4;
-    const int t_tok = ((lane >> 4) << 3) | x7;        // 16-bit V^T matrices: tok half = bit 4
-    const int t_co = (lane >> 3) & 1;
-    const int r = lane >> 2, q4 = lane & 3;
-
-    // ---- S^T = K . Q^T --------------------------------------------------------------------
-    float sc[NT][4];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
     if constexpr (C::kFp8) {
@@ -152,17 +146,34 @@ struct TcMath {
         for (int nt = 0; nt < NT; ++nt) mma_16816<C::kMmaBf16>(sc[nt], a, qf[nt][ks][0], qf[nt][ks][1]);
       }
     }
+  }
 
-    // ---- online softmax over this page (log2 domain) -------------------------------------
-    const bool v_lo = tok_of_row(r) < nv, v_hi = tok_of_row(r + 8) < nv;
-    uint32_t pf[NT][2];
+  // Online softmax (log2 domain) over NP consecutive pages' scores (nv[i] valid tokens each): one
+  // cross-lane max, one raise of the running max and one rescale test for all of them. Returns the
+  // pages' P^T fragments for the P.V products. With NP = 1 this is the per-page step.
+  template <int NP>
+  __device__ __forceinline__ void softmax(const float (&sc)[NP][NT][4], const int (&nv)[NP], float sl2,
+                                          uint32_t (&pf)[NP][NT][2]) {
+    const int r = lane >> 2;
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
-      float s0 = v_lo ? sc[nt][0] * sl2 : -INFINITY;
-      float s1 = v_lo ? sc[nt][1] * sl2 : -INFINITY;
-      float s2 = v_hi ? sc[nt][2] * sl2 : -INFINITY;
-      float s3 = v_hi ? sc[nt][3] * sl2 : -INFINITY;
-      float mx0 = fmaxf(s0, s2), mx1 = fmaxf(s1, s3);
+      float sv[NP][4];
+      float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < NP; ++i) {
+        const bool v_lo = tok_of_row(r) < nv[i], v_hi = tok_of_row(r + 8) < nv[i];
+        sv[i][0] = v_lo ? sc[i][nt][0] * sl2 : -INFINITY;
+        sv[i][1] = v_lo ? sc[i][nt][1] * sl2 : -INFINITY;
+        sv[i][2] = v_hi ? sc[i][nt][2] * sl2 : -INFINITY;
+        sv[i][3] = v_hi ? sc[i][nt][3] * sl2 : -INFINITY;
+        if (i == 0) {
+          mx0 = fmaxf(sv[0][0], sv[0][2]);
+          mx1 = fmaxf(sv[0][1], sv[0][3]);
+        } else {
+          mx0 = fmaxf(mx0, fmaxf(sv[i][0], sv[i][2]));
+          mx1 = fmaxf(mx1, fmaxf(sv[i][1], sv[i][3]));
+        }
+      }
 #pragma unroll
       for (int off = 4; off < 32; off <<= 1) {
         mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, off));
@@ -172,12 +183,25 @@ struct TcMath {
       const float al0 = ex2(m[nt][0] - mn0), al1 = ex2(m[nt][1] - mn1);
       m[nt][0] = mn0;
       m[nt][1] = mn1;
-      const uint32_t x0 = pack2<C::kMmaBf16>(ex2(s0 - mn0), ex2(s1 - mn1));
-      const uint32_t x1 = pack2<C::kMmaBf16>(ex2(s2 - mn0), ex2(s3 - mn1));
       // The denominator sums the same rounded weights the PV product uses.
-      const float2 f0 = unpack2<C::kMmaBf16>(x0), f1 = unpack2<C::kMmaBf16>(x1);
-      l[nt][0] = l[nt][0] * al0 + (f0.x + f1.x);
-      l[nt][1] = l[nt][1] * al1 + (f0.y + f1.y);
+      float ls0 = 0.f, ls1 = 0.f;
+#pragma unroll
+      for (int i = 0; i < NP; ++i) {
+        const uint32_t x0 = pack2<C::kMmaBf16>(ex2(sv[i][0] - mn0), ex2(sv[i][1] - mn1));
+        const uint32_t x1 = pack2<C::kMmaBf16>(ex2(sv[i][2] - mn0), ex2(sv[i][3] - mn1));
+        const float2 f0 = unpack2<C::kMmaBf16>(x0), f1 = unpack2<C::kMmaBf16>(x1);
+        if (i == 0) {
+          ls0 = f0.x + f1.x;
+          ls1 = f0.y + f1.y;
+        } else {
+          ls0 += f0.x + f1.x;
+          ls1 += f0.y + f1.y;
+        }
+        pf[i][nt][0] = movmatrix_trans(x0);  // (k = tok 2q, 2q+1 ; n = g = r)
+        pf[i][nt][1] = movmatrix_trans(x1);  // (k = tok 2q+8, 2q+9)
+      }
+      l[nt][0] = l[nt][0] * al0 + ls0;
+      l[nt][1] = l[nt][1] * al1 + ls1;
       if (__any_sync(kFull, al0 != 1.f || al1 != 1.f)) {  // skipped once the running max settles
 #pragma unroll
         for (int mt = 0; mt < KS; ++mt) {
@@ -187,10 +211,15 @@ struct TcMath {
           acc[nt][mt][3] *= al1;
         }
       }
-      pf[nt][0] = movmatrix_trans(x0);  // (k = tok 2q, 2q+1 ; n = g = r)
-      pf[nt][1] = movmatrix_trans(x1);  // (k = tok 2q+8, 2q+9)
     }
+  }
 
+  // O^T += V^T . P^T of one page (V page at shared address vb, nv valid tokens).
+  __device__ __forceinline__ void pv(uint32_t vb, int nv, const uint32_t (&pf)[NT][2]) {
+    const int x7 = lane & 7;
+    const int t_tok = ((lane >> 4) << 3) | x7;  // 16-bit V^T matrices: tok half = bit 4
+    const int t_co = (lane >> 3) & 1;
+    const int q4 = lane & 3;
     // Tokens past the context may hold any bits (NaN included): zero them in V^T so 0 * NaN
     // never reaches the accumulator. mlo covers k-slots 2q, 2q+1, mhi k-slots 2q+8, 2q+9.
     uint32_t mlo = 0xffffffffu, mhi = 0xffffffffu;
@@ -199,8 +228,6 @@ struct TcMath {
       mlo = (t0 < nv ? 0x0000ffffu : 0u) | (t0 + 1 < nv ? 0xffff0000u : 0u);
       mhi = (t8 < nv ? 0x0000ffffu : 0u) | (t8 + 1 < nv ? 0xffff0000u : 0u);
     }
-
-    // ---- O^T += V^T . P^T -----------------------------------------------------------------
     if constexpr (C::kFp8) {
       // Lanes 0-15 address token rows of chunk 2 mp, lanes 16-31 those of chunk 2 mp + 1 (16 d each);
       // each lane gets tokens 4 q .. 4 q + 3 of d = r and r + 8 of both chunks: k-slots (2q, 2q+1)
@@ -239,6 +266,29 @@ struct TcMath {
         for (int nt = 0; nt < NT; ++nt) mma_16816<C::kMmaBf16>(acc[nt][mt], a, pf[nt][0], pf[nt][1]);
       }
     }
+  }
+
+  // One 16-token page; kb/vb are the shared addresses of its K and V pages; nv valid tokens.
+  __device__ __forceinline__ void page(uint32_t kb, uint32_t vb, int nv, float sl2) {
+    float sc[1][NT][4];
+    qk(kb, sc[0]);
+    uint32_t pf[1][NT][2];
+    const int nvs[1] = {nv};
+    softmax<1>(sc, nvs, sl2, pf);
+    pv(vb, nv, pf[0]);
+  }
+
+  // Two consecutive pages of one partition (A before B in token order) as one softmax step.
+  __device__ __forceinline__ void page2(uint32_t kba, uint32_t vba, int nva, uint32_t kbb, uint32_t vbb, int nvb,
+                                        float sl2) {
+    float sc[2][NT][4];
+    qk(kba, sc[0]);
+    qk(kbb, sc[1]);
+    uint32_t pf[2][NT][2];
+    const int nvs[2] = {nva, nvb};
+    softmax<2>(sc, nvs, sl2, pf);
+    pv(vba, nva, pf[0]);
+    pv(vbb, nvb, pf[1]);
   }
 
   // Zero the running state (a new partition, same query).

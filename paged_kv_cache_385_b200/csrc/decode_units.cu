@@ -249,20 +249,39 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, OCC)
     } else {
       tc.reset();
     }
-    for (int j = 0; j < cu.np; ++j) {
+    // Pages two at a time (one softmax step for both) while the unit has two left, else one.
+    for (int j = 0; j < cu.np;) {
       const int st = consumed % S;
-      const bool got = mbar_wait_bounded(bar0 + 8 * st, (consumed / S) & 1, deadline);
+      const bool pair = j + 1 < cu.np;
+      const int st2 = (consumed + 1) % S;
+      const bool got = mbar_wait_bounded(bar0 + 8 * st, (consumed / S) & 1, deadline) &&
+                       (!pair || mbar_wait_bounded(bar0 + 8 * st2, ((consumed + 1) / S) & 1, deadline));
       if (!__all_sync(kFull, got)) {
         ok = false;
         break;
       }
-      if (meta[warp * S + st]) {
-        const int nv = min(16, cu.ctx_eff - (cu.j0 + j) * 16);
-        tc.page(wbuf_s + st * C::kStageBytes, wbuf_s + st * C::kStageBytes + C::kPageBytes, nv, p.score_scale_log2);
+      const uint32_t ka = wbuf_s + st * C::kStageBytes, kb2 = wbuf_s + st2 * C::kStageBytes;
+      const int nva = min(16, cu.ctx_eff - (cu.j0 + j) * 16);
+      const bool va = meta[warp * S + st] != 0;
+      if (pair) {
+        const int nvb = min(16, cu.ctx_eff - (cu.j0 + j + 1) * 16);
+        const bool vb = meta[warp * S + st2] != 0;
+        if (va && vb) {
+          tc.page2(ka, ka + C::kPageBytes, nva, kb2, kb2 + C::kPageBytes, nvb, p.score_scale_log2);
+        } else {  // a page skipped for a bad block id (already reported)
+          if (va) tc.page(ka, ka + C::kPageBytes, nva, p.score_scale_log2);
+          if (vb) tc.page(kb2, kb2 + C::kPageBytes, nvb, p.score_scale_log2);
+        }
+      } else if (va) {
+        tc.page(ka, ka + C::kPageBytes, nva, p.score_scale_log2);
       }
       __syncwarp();
-      ++consumed;
-      issue_next();
+      const int n = pair ? 2 : 1;
+      for (int i = 0; i < n; ++i) {
+        ++consumed;
+        issue_next();
+      }
+      j += n;
     }
     if (!ok) break;
     tc.template write_global<C::kQBf16>(p, cu.s, cu.hk, cu.part, !p.always_partials && cu.nparts <= 1, keep_pol);
