@@ -69,6 +69,8 @@ CASES = [
     # Groups of 16 query heads (the largest the tcgen05 kernel takes: 8 tokens x 16 heads per tile),
     # chunks that end mid-tile, one sequence with a single new token.
     ([333, 70, 1], [101, 70, 1], 32, 2, 128, torch.float16),
+    # A sequence with no new tokens in the batch (its items have no rows).
+    ([50, 300, 10], [0, 200, 10], 8, 2, 128, torch.bfloat16),
 ]
 
 
@@ -107,6 +109,21 @@ def test_prefill_scale_sign_and_size(scale, kernel):
     want = _oracle(host, q, qs, ctxs, scale, hkv, "f16")
     err = float(np.max(np.abs(out.double().cpu().numpy() - want)))
     assert err <= TOL["f16"], err
+
+
+@pytest.mark.parametrize("kernel", [0, 1])
+def test_prefill_with_a_loose_max_query_len(kernel):
+    """max_query_len is only a bound: twice the real one sizes a grid whose later row tiles have no rows
+    in any sequence (the persistent kernel's CTAs skip those items, every role alike)."""
+    ctxs, news, hq, hkv, d, dtype = [700, 260, 1300], [400, 131, 64], 32, 8, 128, torch.bfloat16
+    bt, kc, vc, q, qs, host = _build(ctxs, news, hq, hkv, d, dtype, seed=88)
+    out = torch.full((q.shape[0], hq, d), float("nan"), dtype=dtype, device="cuda")
+    pa.pa_prefill(out, q.cuda(), kc, vc, bt.cuda(), qs.cuda(), torch.tensor(ctxs, dtype=torch.int32).cuda(),
+                  2 * max(news), d ** -0.5, hkv, kernel=kernel)
+    torch.cuda.synchronize()
+    assert pa.pa_read_device_error(clear=True) == 0
+    want = _oracle(host, q, qs, ctxs, d ** -0.5, hkv, "bf16")
+    assert float(np.max(np.abs(out.double().cpu().numpy() - want))) <= TOL["bf16"]
 
 
 def test_tcgen05_and_warp_mma_prefill_agree():
