@@ -31,7 +31,7 @@ namespace pa {
 namespace {
 
 constexpr int kD = 128;
-constexpr int kRows = 128;   // query rows per CTA
+constexpr int kRows = 128;   // query rows per work item
 constexpr int kThreads = 256;
 constexpr uint32_t kHalf = 16384;  // one 64-element (128-byte) column half of a 128-row tile
 constexpr uint32_t kTile = 2 * kHalf;
