@@ -302,8 +302,10 @@ def ncu_traffic(workload: str):
         return None
 
 
-def cpu_baseline_sample(w: W.Workload, budget_s: float = 15.0):
-    """Time the float64 oracle (as it stands) on whole sequences of the workload until ~budget_s."""
+def cpu_baseline_sample(w: W.Workload, budget_s: float = 15.0, min_s: float = 10.0):
+    """Time the float64 oracle (as it stands) on whole sequences of the workload: at least min_s of
+    oracle time (passing over the batch again when it finishes sooner), and no new sequence after
+    budget_s once every sequence has run once."""
     import numpy as np
     from oracle import attention
     try:
@@ -315,7 +317,19 @@ def cpu_baseline_sample(w: W.Workload, budget_s: float = 15.0):
     rng = np.random.default_rng(w.seed)
     D, Hkv, Hq = w.head_dim, w.num_kv_heads, w.num_q_heads
     esz = w.kv_elem_bytes
-    done_bytes, t_total, nseq = 0, 0.0, 0
+    done_bytes, t_total, nseq, done_tokens = 0, 0.0, 0, 0
+    kept, kept_bytes = [], 0  # the first pass's inputs (up to 256 MB of pools) for the repeat passes
+
+    def timed(args):
+        nonlocal done_bytes, t_total, nseq, done_tokens
+        q, kp, vp, bt, n = args
+        t0 = time.perf_counter()
+        attention.decode_paged(q, kp, vp, bt, [n], w.scale, Hkv, w.kv_dtype, 0.0123, 0.0123)
+        t_total += time.perf_counter() - t0
+        done_bytes += n * Hkv * D * esz * 2
+        done_tokens += n
+        nseq += 1
+
     while nseq == 0 or (t_total < budget_s and nseq < w.num_seqs):
         n = int(lens[nseq])
         nb = -(-n // 16)
@@ -328,13 +342,18 @@ def cpu_baseline_sample(w: W.Workload, budget_s: float = 15.0):
             vp = torch.randn(nb, Hkv, 16, D).to(tdt).view(torch.int16).numpy().view(np.uint8)
         bt = rng.permutation(nb).astype(np.int32)[None, :]
         q = rng.standard_normal((1, Hq, D))
-        t0 = time.perf_counter()
-        attention.decode_paged(q, kp, vp, bt, [n], w.scale, Hkv, w.kv_dtype, 0.0123, 0.0123)
-        t_total += time.perf_counter() - t0
-        done_bytes += n * Hkv * D * esz * 2
-        nseq += 1
+        if kept_bytes + 2 * kp.nbytes <= (256 << 20):
+            kept.append((q, kp, vp, bt, n))
+            kept_bytes += 2 * kp.nbytes
+        timed((q, kp, vp, bt, n))
+    while t_total < min_s and kept:  # repeat passes over the kept sequences until min_s of oracle time
+        for args in kept:
+            timed(args)
+    what = (f"{nseq} of {w.num_seqs} sequences" if nseq <= w.num_seqs else
+            f"{nseq} sequence runs (each of the {w.num_seqs} sequences once, then repeats over the first "
+            f"{len(kept)} until {min_s:.0f} s of oracle time)")
     return {"value": done_bytes / t_total / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
-            "sample": f"{nseq} of {w.num_seqs} sequences (all {Hq} query heads, {int(lens[:nseq].sum())} tokens), "
+            "sample": f"{what} (all {Hq} query heads, {done_tokens} tokens), "
                       f"float64 numpy oracle (gather through the block table + softmax(qK^T)V), "
                       f"{t_total:.1f} s wall"}
 
@@ -560,7 +579,7 @@ def run_reference(args, rank, world):
     per_step = []
     cpu = None
     for i in range(max(3, args.warmup) + args.steps):
-        r = cpu_baseline_sample(w, budget_s=0.0)  # one sequence per step
+        r = cpu_baseline_sample(w, budget_s=0.0, min_s=0.0)  # one sequence per step
         if i >= max(3, args.warmup):
             per_step.append(r)
         cpu = r
